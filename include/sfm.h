@@ -1,0 +1,228 @@
+/*
+ * sfm.h -- C ABI of libsfm: the batch-folded Mamba selective scan of SF-Mamba on B200.
+ *
+ * The operation (per sample b, channel d, within-sample token t = 0..L-1):
+ *
+ *   xa      = [avg(x), x_1 .. x_T, avg(x)]              stage-entry layer only (aux init)
+ *   u_t     = SiLU(conv_b + sum_k conv_w[k] * xa[t + k - pad_left])   zero outside the sample
+ *   Delta_t = softplus(dt_t + dt_bias)
+ *   Abar_tn = exp(Delta_t * A_n), except Abar = 0 at every sample start (the reset)
+ *   h_tn    = Abar_tn * h_(t-1)n + Delta_t * B_tn * u_t
+ *   y_t     = (sum_n C_tn * h_tn + Dskip * u_t) * SiLU(z_t)
+ *   out     = y with tokens 0 and L-1 exchanged (aux swap), when requested.
+ *
+ * Passages this follows:
+ *   - recurrence h_t = Abar_t h_{t-1} + Bbar_t x_t, y_t = C_t h_t:
+ *     "SF-Mamba: Scan Folding" (sungsoo.github.io), section 3.1;
+ *   - aux head/tail tokens initialised to avg(X), swapped head<->tail between layers:
+ *     same page, section 3.2 equations; "SF-Mamba: Rethinking Vision Mamba"
+ *     (techloop.online), Auxiliary Patch Swapping;
+ *   - folding [B,D,T] -> [B1,D,B2*T], B = B1*B2, with Abar_t = 0 at every sample start:
+ *     sungsoo.github.io section 3.3 equations; techloop.online, Batch Folding with
+ *     Periodic State Reset;
+ *   - a conv that never crosses folded sample boundaries: techloop.online, the
+ *     convolution-boundary paragraph; sungsoo.github.io section 8.1 item 5;
+ *   - B1 chosen from an offline look-up table: techloop.online, Adaptive B1;
+ *     sungsoo.github.io section 8.1 item 6.
+ *   The discretisation (Abar = exp(Delta*A), Bbar = Delta*B), the D skip, softplus and
+ *   the SiLU(z) gate are the standard Mamba block; the pages do not spell them out.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library never
+ *     allocates device memory, never frees it, and never synchronises the stream
+ *     (sfm_get_device_error is the one documented exception).
+ *   - Layouts are contiguous row-major: x [B,D,T] (aux init) or [B,D,L]; dt, z, y
+ *     [B,D,L]; Bm, Cm [B,N,L] (one group shared by all channels); A [D,N];
+ *     Dskip, dt_bias, conv_b [D]; conv_w [D,K]; final_state [B,D,N].
+ *   - Activation tensors are fp32 or bf16 (sfm_dtype); parameters are always fp32;
+ *     the state and every accumulation are fp32 on the device.
+ *   - Argument errors are reported synchronously, before anything is launched, and
+ *     leave the device untouched. A launch failure returns SFM_ERR_CUDA.
+ *   - Work is enqueued on `stream` (NULL = the legacy default stream).
+ *   - Setting the environment variable SFM_FAULT_INJECT=launch makes every compute
+ *     entry point return SFM_ERR_CUDA after validation without launching (host-side
+ *     fault injection for tests; nothing reaches the GPU).
+ */
+#ifndef SFM_H
+#define SFM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Entry points are the only symbols the shared library exports. */
+#if defined(__GNUC__)
+#define SFM_API __attribute__((visibility("default")))
+#else
+#define SFM_API
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* sfm_stream_t;
+
+typedef enum {
+  SFM_OK = 0,
+  SFM_ERR_INVALID_ARG = 1, /* NULL where a tensor is required, bad size or flag     */
+  SFM_ERR_MISALIGNED = 2,  /* a tensor base pointer is not 16-byte aligned          */
+  SFM_ERR_UNSUPPORTED = 3, /* valid but outside what the kernels cover (N, K, ...)   */
+  SFM_ERR_CUDA = 4,        /* the CUDA runtime reported an error at launch           */
+  SFM_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (device error word)    */
+} sfm_status;
+
+typedef enum { SFM_F32 = 0, SFM_BF16 = 1 } sfm_dtype;
+
+/* Largest supported sizes. */
+#define SFM_MAX_N 64      /* state size                                     */
+#define SFM_MAX_K 4       /* conv width                                     */
+#define SFM_MAX_L 16384   /* tokens per sample (aux tokens included)        */
+
+/* Human-readable name of a status code; never NULL. */
+SFM_API const char* sfm_status_string(int status);
+
+/* ABI version (bumped on any change of a struct layout or signature). */
+SFM_API int sfm_abi_version(void);
+
+/* Name of the CUDA error behind the calling thread's most recent SFM_ERR_CUDA
+ * ("none" if there was none); the string is static. */
+SFM_API const char* sfm_last_cuda_error(void);
+
+/*
+ * Aux init (stage-entry layer): xa[b,d,0] = xa[b,d,T+1] = mean_t x[b,d,t] (fp32 sum),
+ * xa[b,d,1..T] = x[b,d,0..T-1].  x [B,D,T] -> xa [B,D,T+2], both `dtype`.
+ * Source: techloop.online, Auxiliary Patch Swapping (avg(X) initialisation);
+ * sungsoo.github.io section 3.2.  x and xa must not overlap.
+ */
+SFM_API sfm_status sfm_aux_init(const void* x, void* xa, int B, int D, int T, sfm_dtype dtype,
+                        sfm_stream_t stream);
+
+/*
+ * Aux swap between consecutive layers, in place: y[b,d,0] <-> y[b,d,L-1].  L >= 2.
+ * Source: sungsoo.github.io section 3.2 (next head = this tail, next tail = this head).
+ */
+SFM_API sfm_status sfm_aux_swap(void* y, int B, int D, int L, sfm_dtype dtype, sfm_stream_t stream);
+
+/*
+ * Boundary-safe depthwise conv1d on the folded layout:
+ *   u[b,d,t] = act(bias[d] + sum_{k<K} w[d,k] * x[b,d,t+k-pad_left]),
+ * with zeros wherever t+k-pad_left falls outside [0,L) of sample b -- a folded row of
+ * B2 samples is never read across a sample boundary.  act = SiLU if silu != 0.
+ * x, u [B,D,L] (`dtype`, must not overlap); w [D,K] fp32; bias [D] fp32 or NULL.
+ * 1 <= K <= SFM_MAX_K, 0 <= pad_left < K; B2 >= 1 must divide B (the result does not
+ * depend on B2).  Source: techloop.online convolution-boundary paragraph;
+ * sungsoo.github.io section 8.1 item 5.
+ */
+SFM_API sfm_status sfm_fold_conv1d(const void* x, const float* w, const float* bias, void* u,
+                           int B, int D, int L, int K, int pad_left, int B2, int silu,
+                           sfm_dtype dtype, sfm_stream_t stream);
+
+/* Arguments of the fused folded scan.  `size` must be sizeof(sfm_scan_args). */
+typedef struct {
+  uint32_t size;
+  /* activations (in_dtype) */
+  const void* x;        /* conv input: [B,D,L-2] if aux_init else [B,D,L]; with
+                           conv_w == NULL it is the scan input u itself            */
+  const void* dt;       /* [B,D,L] raw Delta before bias/softplus                  */
+  const void* z;        /* [B,D,L] gate input, or NULL for no gate                 */
+  const void* Bm;       /* [B,N,L]                                                 */
+  const void* Cm;       /* [B,N,L]                                                 */
+  /* parameters (fp32) */
+  const float* A;       /* [D,N]                                                   */
+  const float* Dskip;   /* [D] or NULL                                             */
+  const float* dt_bias; /* [D] or NULL                                             */
+  const float* conv_w;  /* [D,K] or NULL (no conv: x is u)                         */
+  const float* conv_b;  /* [D] or NULL                                             */
+  /* outputs */
+  void* y;              /* [B,D,L] out_dtype; must not overlap any input          */
+  float* final_state;   /* [B,D,N] fp32 state after each sample's last token, or NULL */
+  /* sizes */
+  int B, D, L, N;
+  int K, pad_left;      /* conv width and left padding (used when conv_w != NULL)  */
+  int B1;               /* folded rows; 0 = choose with sfm_choose_b1; must divide B */
+  int reset_period;     /* 0 or L: the state restarts every L folded positions     */
+  /* flags */
+  int dt_softplus;      /* Delta = softplus(dt + dt_bias) if set, else dt + dt_bias */
+  int aux_init;         /* x holds T = L-2 tokens; build the aux tokens on load    */
+  int swap_out;         /* exchange output tokens 0 and L-1 on store               */
+  sfm_dtype in_dtype, out_dtype; /* (F32,F32), (BF16,BF16) or (BF16,F32)           */
+  /* launch shape overrides for sweeps; 0 = automatic */
+  int lanes;            /* lanes per channel sequence (1 = one thread walks it)    */
+  int d_tile;           /* channels per CTA (at most 128)                          */
+  int chunk;            /* tokens staged per step of the walk                      */
+} sfm_scan_args;
+
+/*
+ * The fused forward of the hot path: [aux init] -> conv + SiLU -> Delta -> folded
+ * scan with reset -> D skip -> SiLU(z) gate -> [aux swap], one kernel launch.
+ * Samples are grouped into B1 folded rows of B2 = B/B1 samples; each CTA walks the
+ * B2 samples of one row for a tile of channels, restarting the state at every
+ * sample start.  The result is independent of B1 (the reset makes the samples
+ * independent), so B1 only changes the schedule.
+ * Requirements: x, dt, z, Bm, Cm, y 16-byte aligned; 1 <= N <= SFM_MAX_N;
+ * 1 <= K <= SFM_MAX_K; 3 <= L <= SFM_MAX_L when aux_init (else 1 <= L); y must not
+ * alias an input.  Sources: see the header comment.
+ */
+SFM_API sfm_status sfm_selective_scan_fold(const sfm_scan_args* args, sfm_stream_t stream);
+
+/* Gradients produced by the scan backward (all fp32, caller-owned device memory). */
+typedef struct {
+  uint32_t size;        /* sizeof(sfm_scan_grads)                                 */
+  const void* dout;     /* [B,D,L] upstream gradient of y, args->out_dtype        */
+  float* du;            /* [B,D,L]                                                */
+  float* ddt;           /* [B,D,L]  (through the softplus when dt_softplus)       */
+  float* dz;            /* [B,D,L]  or NULL when args->z is NULL                  */
+  float* dA;            /* [D,N]    summed over samples and tokens                */
+  float* dDskip;        /* [D]      or NULL when args->Dskip is NULL              */
+  float* ddt_bias;      /* [D]      or NULL when args->dt_bias is NULL            */
+  float* dB;            /* [B,N,L]  summed over channels                          */
+  float* dC;            /* [B,N,L]  summed over channels                          */
+} sfm_scan_grads;
+
+/*
+ * Workspace (bytes) the scan backward needs for `args`; 256-byte aligned device
+ * memory of at least this size goes to sfm_selective_scan_fold_bwd.
+ */
+SFM_API sfm_status sfm_scan_bwd_workspace_size(const sfm_scan_args* args, size_t* bytes);
+
+/*
+ * Backward of the scan (from its input u to the gated output): a reverse adjoint
+ * sweep g_t = C_t dy_t + Abar_(t+1) g_(t+1) that never crosses a sample start, where
+ * the transition factor is the constant 0.  Reductions over channels (dB, dC) and
+ * over samples/tokens (dA, dDskip, ddt_bias) are done in a fixed order, so results
+ * are bitwise reproducible.  args must describe a scan without conv, aux init or
+ * swap (conv_w == NULL, aux_init == 0, swap_out == 0); args->y is not read.
+ * Overwrites every gradient buffer given.  Source: the reset reading of
+ * sungsoo.github.io section 3.3; the backward itself is not on the pages.
+ */
+SFM_API sfm_status sfm_selective_scan_fold_bwd(const sfm_scan_args* args, const sfm_scan_grads* grads,
+                                       void* workspace, size_t workspace_bytes,
+                                       sfm_stream_t stream);
+
+/*
+ * Adaptive B1: the number of folded rows for a batch of B samples of T patch tokens,
+ * D channels and state size N, from a look-up table built by a B200 sweep.  The
+ * result always divides B.  Source: techloop.online, Adaptive B1; sungsoo.github.io
+ * section 8.1 item 6.  Pure host function.
+ */
+SFM_API sfm_status sfm_choose_b1(int B, int T, int D, int N, int* B1_out);
+
+/* The full launch choice behind sfm_choose_b1: folded rows, lanes per channel
+ * sequence, channels per CTA and tokens staged per step. */
+typedef struct {
+  int B1, lanes, d_tile, chunk;
+} sfm_variant;
+SFM_API sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* out);
+
+/*
+ * Reads (and, if clear != 0, resets) the device-side error word that kernels set when
+ * a bounded wait gives up.  Synchronises `stream` first.  *code = SFM_OK when clean.
+ */
+SFM_API sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFM_H */

@@ -1,0 +1,206 @@
+"""selective_scan_sfm_b200 -- the batch-folded selective scan of SF-Mamba on B200.
+
+A thin PyTorch-facing binding over the C ABI in include/sfm.h (libsfm.so, hand-written
+sm_100a CUDA).  Every function here only checks and marshals arguments: all steps of
+the path run inside the library's kernels; PyTorch provides device memory and streams.
+Names follow the C entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _abi
+from ._abi import SFM_BF16, SFM_F32, SfmError
+
+__all__ = [
+    "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d", "sfm_selective_scan_fold",
+    "sfm_selective_scan_fold_bwd", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
+    "SfmError", "library_path",
+]
+
+_DT = {torch.float32: SFM_F32, torch.bfloat16: SFM_BF16}
+
+
+def library_path() -> str:
+    return _abi.LIB_PATH
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, name, dtype=None, shape=None, optional=False):
+    if t is None:
+        if optional:
+            return None
+        raise ValueError("%s is required" % name)
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _code(dtype) -> int:
+    if dtype not in _DT:
+        raise ValueError("unsupported dtype %s (float32 or bfloat16)" % dtype)
+    return _DT[dtype]
+
+
+def sfm_aux_init(x, xa=None, stream=None):
+    """x [B,D,T] -> xa [B,D,T+2] with head = tail = mean over the T tokens."""
+    _dev(x, "x")
+    B, D, T = x.shape
+    if xa is None:
+        xa = torch.empty(B, D, T + 2, dtype=x.dtype, device=x.device)
+    _dev(xa, "xa", x.dtype, (B, D, T + 2))
+    _abi.check(_abi.lib().sfm_aux_init(_ptr(x), _ptr(xa), B, D, T, _code(x.dtype), _stream(stream)), "sfm_aux_init")
+    return xa
+
+
+def sfm_aux_swap(y, stream=None):
+    """In place: y[..., 0] <-> y[..., L-1]."""
+    _dev(y, "y")
+    B, D, L = y.shape
+    _abi.check(_abi.lib().sfm_aux_swap(_ptr(y), B, D, L, _code(y.dtype), _stream(stream)), "sfm_aux_swap")
+    return y
+
+
+def sfm_fold_conv1d(x, w, bias=None, u=None, pad_left=None, B2=1, silu=False, stream=None):
+    """Depthwise conv1d with zero padding per sample; x, u [B,D,L]; w [D,K] fp32."""
+    _dev(x, "x")
+    B, D, L = x.shape
+    _dev(w, "w", torch.float32)
+    K = w.shape[1]
+    _dev(w, "w", torch.float32, (D, K))
+    _dev(bias, "bias", torch.float32, (D,), optional=True)
+    if u is None:
+        u = torch.empty_like(x)
+    _dev(u, "u", x.dtype, (B, D, L))
+    pl = (K - 1) // 2 if pad_left is None else int(pad_left)
+    _abi.check(_abi.lib().sfm_fold_conv1d(_ptr(x), _ptr(w), _ptr(bias), _ptr(u), B, D, L, K, pl, int(B2),
+                                          int(bool(silu)), _code(x.dtype), _stream(stream)), "sfm_fold_conv1d")
+    return u
+
+
+def _scan_args(x, dt, Bm, Cm, A, z, Dskip, dt_bias, conv_w, conv_b, y, final_state, B1, pad_left, dt_softplus,
+               aux_init, swap_out, out_dtype, lanes, d_tile, chunk, need_y=True):
+    _dev(dt, "dt")
+    B, D, L = dt.shape
+    io = dt.dtype
+    T = L - 2 if aux_init else L
+    _dev(x, "x", io, (B, D, T))
+    N = Bm.shape[1] if isinstance(Bm, torch.Tensor) and Bm.dim() == 3 else -1
+    _dev(Bm, "Bm", io, (B, N, L))
+    _dev(Cm, "Cm", io, (B, N, L))
+    _dev(z, "z", io, (B, D, L), optional=True)
+    _dev(A, "A", torch.float32, (D, N))
+    _dev(Dskip, "Dskip", torch.float32, (D,), optional=True)
+    _dev(dt_bias, "dt_bias", torch.float32, (D,), optional=True)
+    K = 0
+    if conv_w is not None:
+        _dev(conv_w, "conv_w", torch.float32)
+        K = conv_w.shape[1]
+        _dev(conv_w, "conv_w", torch.float32, (D, K))
+    _dev(conv_b, "conv_b", torch.float32, (D,), optional=True)
+    od = io if out_dtype is None else out_dtype
+    if need_y:
+        if y is None:
+            y = torch.empty(B, D, L, dtype=od, device=dt.device)
+        _dev(y, "y", od, (B, D, L))
+    _dev(final_state, "final_state", torch.float32, (B, D, N), optional=True)
+    a = _abi.ScanArgs()
+    a.size = ctypes.sizeof(_abi.ScanArgs)
+    a.x, a.dt, a.z, a.Bm, a.Cm = (t.data_ptr() if t is not None else None for t in (x, dt, z, Bm, Cm))
+    a.A, a.Dskip, a.dt_bias, a.conv_w, a.conv_b = (t.data_ptr() if t is not None else None
+                                                   for t in (A, Dskip, dt_bias, conv_w, conv_b))
+    a.y = y.data_ptr() if y is not None else None
+    a.final_state = final_state.data_ptr() if final_state is not None else None
+    a.B, a.D, a.L, a.N = B, D, L, N
+    a.K = K
+    a.pad_left = ((K - 1) // 2 if pad_left is None else int(pad_left)) if K else 0
+    a.B1 = int(B1)
+    a.reset_period = L
+    a.dt_softplus, a.aux_init, a.swap_out = int(bool(dt_softplus)), int(bool(aux_init)), int(bool(swap_out))
+    a.in_dtype, a.out_dtype = _code(io), _code(od)
+    a.lanes, a.d_tile, a.chunk = int(lanes), int(d_tile), int(chunk)
+    return a, y
+
+
+def sfm_selective_scan_fold(x, dt, Bm, Cm, A, *, z=None, Dskip=None, dt_bias=None, conv_w=None, conv_b=None,
+                            y=None, final_state=None, B1=0, pad_left=None, dt_softplus=True, aux_init=False,
+                            swap_out=False, out_dtype=None, lanes=0, d_tile=0, chunk=0, stream=None):
+    """Fused forward: [aux init] -> conv+SiLU -> folded scan with reset -> D skip ->
+    SiLU(z) gate -> [aux swap].  Returns y [B,D,L]."""
+    a, y = _scan_args(x, dt, Bm, Cm, A, z, Dskip, dt_bias, conv_w, conv_b, y, final_state, B1, pad_left,
+                      dt_softplus, aux_init, swap_out, out_dtype, lanes, d_tile, chunk)
+    _abi.check(_abi.lib().sfm_selective_scan_fold(ctypes.byref(a), _stream(stream)), "sfm_selective_scan_fold")
+    return y
+
+
+def sfm_selective_scan_fold_bwd(u, dt, Bm, Cm, A, dout, *, z=None, Dskip=None, dt_bias=None, B1=0,
+                                dt_softplus=True, workspace=None, grads=None, stream=None):
+    """Backward of the gated scan (input u, no conv).  Returns a dict of fp32 grads."""
+    a, _ = _scan_args(u, dt, Bm, Cm, A, z, Dskip, dt_bias, None, None, None, None, B1, None, dt_softplus,
+                      False, False, None, 0, 0, 0, need_y=False)
+    B, D, L, N = a.B, a.D, a.L, a.N
+    _dev(dout, "dout", dt.dtype, (B, D, L))
+    dev = dt.device
+    f32 = torch.float32
+    if grads is None:
+        grads = dict(du=torch.empty(B, D, L, dtype=f32, device=dev), ddt=torch.empty(B, D, L, dtype=f32, device=dev),
+                     dA=torch.empty(D, N, dtype=f32, device=dev), dB=torch.empty(B, N, L, dtype=f32, device=dev),
+                     dC=torch.empty(B, N, L, dtype=f32, device=dev))
+        if z is not None:
+            grads["dz"] = torch.empty(B, D, L, dtype=f32, device=dev)
+        if Dskip is not None:
+            grads["dDskip"] = torch.empty(D, dtype=f32, device=dev)
+        if dt_bias is not None:
+            grads["ddt_bias"] = torch.empty(D, dtype=f32, device=dev)
+    g = _abi.ScanGrads()
+    g.size = ctypes.sizeof(_abi.ScanGrads)
+    g.dout = dout.data_ptr()
+    for k in ("du", "ddt", "dz", "dA", "dDskip", "ddt_bias", "dB", "dC"):
+        t = grads.get(k)
+        setattr(g, k, None if t is None else _dev(t, k, f32).data_ptr())
+    need = ctypes.c_size_t(0)
+    _abi.check(_abi.lib().sfm_scan_bwd_workspace_size(ctypes.byref(a), ctypes.byref(need)),
+               "sfm_scan_bwd_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(int(need.value), 1), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8)
+    _abi.check(_abi.lib().sfm_selective_scan_fold_bwd(ctypes.byref(a), ctypes.byref(g),
+                                                      ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+                                                      _stream(stream)), "sfm_selective_scan_fold_bwd")
+    return grads
+
+
+def sfm_choose_variant(B: int, T: int, D: int, N: int) -> dict:
+    v = _abi.Variant()
+    _abi.check(_abi.lib().sfm_choose_variant(int(B), int(T), int(D), int(N), ctypes.byref(v)), "sfm_choose_variant")
+    return dict(B1=v.B1, lanes=v.lanes, d_tile=v.d_tile, chunk=v.chunk)
+
+
+def sfm_choose_b1(B: int, T: int, D: int, N: int) -> int:
+    out = ctypes.c_int(0)
+    _abi.check(_abi.lib().sfm_choose_b1(int(B), int(T), int(D), int(N), ctypes.byref(out)), "sfm_choose_b1")
+    return out.value
+
+
+def sfm_get_device_error(clear: bool = True, stream=None) -> int:
+    code = ctypes.c_int(0)
+    _abi.check(_abi.lib().sfm_get_device_error(_stream(stream), int(bool(clear)), ctypes.byref(code)),
+               "sfm_get_device_error")
+    return code.value

@@ -1,0 +1,299 @@
+// sfm_api.cu -- the C ABI of libsfm (declared in include/sfm.h): argument validation,
+// the adaptive-B1 chooser, and dispatch to the sm_100a kernels.
+//
+// Validation is complete before any CUDA call, so every argument error returns
+// synchronously and leaves the device untouched.  The library keeps no mutable state
+// besides the once-per-kernel shared-memory attribute and the device error word.
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include "sfm.h"
+#include "sfm_internal.h"
+
+using namespace sfm;
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+constexpr int kMaxDTile = 128;
+constexpr int kMaxChunk = 256;
+constexpr int kMaxB1 = 65535;  // grid.y
+constexpr int kMaxNFused = 16;
+constexpr int kWholeSmemCap = 80 * 1024;  // whole-sample staging only while 2+ CTAs fit an SM
+
+struct LutEntry {
+  int T, B, D, N, B2, lanes, d_tile, chunk;
+};
+const LutEntry kLut[] = {
+#include "sfm_lut.inc"
+};
+
+thread_local const char* t_last_cuda_error = "none";
+
+// Maps a launch result to a status, remembering the CUDA error name for sfm_last_cuda_error.
+sfm_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SFM_OK;
+  t_last_cuda_error = cudaGetErrorName(e);
+  return SFM_ERR_CUDA;
+}
+
+bool fault_injected() {
+  const char* v = std::getenv("SFM_FAULT_INJECT");
+  return v && std::strcmp(v, "launch") == 0;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int esize_of(sfm_dtype t) { return t == SFM_F32 ? 4 : 2; }
+bool dtype_ok(int t) { return t == SFM_F32 || t == SFM_BF16; }
+
+bool overlaps(const void* a, long long abytes, const void* b, long long bbytes) {
+  if (!a || !b) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + (uintptr_t)bbytes && b0 < a0 + (uintptr_t)abytes;
+}
+
+int largest_divisor_at_most(int B, int cap) {
+  if (cap < 1) cap = 1;
+  for (int v = cap < B ? cap : B; v >= 1; --v)
+    if (B % v == 0) return v;
+  return 1;
+}
+
+int round_up(int v, int m) { return (v + m - 1) / m * m; }
+
+// Chunk length: at most `cap` tokens, balanced so that the last chunk is not a sliver,
+// rounded up to a multiple of 8.
+int balanced_chunk(int L, int cap) {
+  const int n = (L + cap - 1) / cap;
+  return round_up((L + n - 1) / n, 8);
+}
+
+// Nearest table row in log space of (T, B*D, N), then adapted to the actual sizes.
+sfm_variant choose(int B, int T, int D, int N) {
+  const LutEntry* best = &kLut[0];
+  double bestd = 1e300;
+  for (const LutEntry& e : kLut) {
+    const double dT = std::log2((double)T / e.T), dW = std::log2((double)B * D / ((double)e.B * e.D)),
+                 dN = std::log2((double)N / e.N);
+    const double dist = 4.0 * dT * dT + dW * dW + 2.0 * dN * dN;
+    if (dist < bestd) {
+      bestd = dist;
+      best = &e;
+    }
+  }
+  sfm_variant v;
+  int B2 = largest_divisor_at_most(B, best->B2);
+  while (B / B2 > kMaxB1) {  // more samples per folded row until the grid fits
+    int next = B2 + 1;
+    while (B % next) ++next;
+    B2 = next;
+  }
+  v.B1 = B / B2;
+  v.lanes = 1;
+  int dt = best->d_tile;
+  if (dt > round_up(D, 32)) dt = round_up(D, 32);
+  v.d_tile = dt;
+  v.chunk = balanced_chunk(T + 2, best->chunk);
+  return v;
+}
+
+sfm_status validate_scan(const sfm_scan_args* a, bool bwd) {
+  if (!a || a->size != sizeof(sfm_scan_args)) return SFM_ERR_INVALID_ARG;
+  if (!a->x || !a->dt || !a->Bm || !a->Cm || !a->A) return SFM_ERR_INVALID_ARG;
+  if (!bwd && !a->y) return SFM_ERR_INVALID_ARG;
+  if (a->B < 1 || a->D < 1 || a->L < 1 || a->N < 1) return SFM_ERR_INVALID_ARG;
+  if (a->N > SFM_MAX_N || a->L > SFM_MAX_L) return SFM_ERR_UNSUPPORTED;
+  if (a->N > kMaxNFused) return SFM_ERR_UNSUPPORTED;
+  if ((a->dt_softplus | a->aux_init | a->swap_out) & ~1) return SFM_ERR_INVALID_ARG;
+  if (a->aux_init && a->L < 3) return SFM_ERR_INVALID_ARG;
+  if (a->conv_w && (a->K < 1 || a->K > SFM_MAX_K || a->pad_left < 0 || a->pad_left >= a->K))
+    return SFM_ERR_INVALID_ARG;
+  if (a->B1 < 0 || (a->B1 > 0 && a->B % a->B1 != 0)) return SFM_ERR_INVALID_ARG;
+  if (a->B1 > kMaxB1) return SFM_ERR_UNSUPPORTED;
+  if (a->reset_period != 0 && a->reset_period != a->L) return SFM_ERR_UNSUPPORTED;
+  if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SFM_ERR_INVALID_ARG;
+  if (a->in_dtype == SFM_F32 && a->out_dtype == SFM_BF16) return SFM_ERR_UNSUPPORTED;
+  if (a->lanes < 0 || a->lanes > 1) return SFM_ERR_UNSUPPORTED;
+  if (a->d_tile < 0 || a->d_tile > kMaxDTile) return SFM_ERR_UNSUPPORTED;
+  if (a->chunk < 0 || a->chunk > kMaxChunk || (a->chunk % 8) != 0) return SFM_ERR_UNSUPPORTED;
+  const void* acts[] = {a->x, a->dt, a->z, a->Bm, a->Cm, a->y};
+  for (const void* p : acts)
+    if (p && !aligned16(p)) return SFM_ERR_MISALIGNED;
+  const long long si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);
+  const long long bdl = (long long)a->B * a->D * a->L;
+  const long long xbytes = (long long)a->B * a->D * (a->aux_init ? a->L - 2 : a->L) * si;
+  const long long bcbytes = (long long)a->B * a->N * a->L * si;
+  if (!bwd) {
+    const long long ybytes = bdl * so;
+    if (overlaps(a->y, ybytes, a->x, xbytes) || overlaps(a->y, ybytes, a->dt, bdl * si) ||
+        overlaps(a->y, ybytes, a->z, bdl * si) || overlaps(a->y, ybytes, a->Bm, bcbytes) ||
+        overlaps(a->y, ybytes, a->Cm, bcbytes))
+      return SFM_ERR_INVALID_ARG;
+  }
+  return SFM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sfm_status_string(int status) {
+  switch (status) {
+    case SFM_OK: return "SFM_OK";
+    case SFM_ERR_INVALID_ARG: return "SFM_ERR_INVALID_ARG: invalid argument";
+    case SFM_ERR_MISALIGNED: return "SFM_ERR_MISALIGNED: tensor base not 16-byte aligned";
+    case SFM_ERR_UNSUPPORTED: return "SFM_ERR_UNSUPPORTED: outside the supported sizes";
+    case SFM_ERR_CUDA: return "SFM_ERR_CUDA: CUDA launch error";
+    case SFM_ERR_TIMEOUT: return "SFM_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    default: return "SFM_ERR_UNKNOWN";
+  }
+}
+
+int sfm_abi_version(void) { return kAbiVersion; }
+
+const char* sfm_last_cuda_error(void) { return t_last_cuda_error; }
+
+sfm_status sfm_aux_init(const void* x, void* xa, int B, int D, int T, sfm_dtype dtype, sfm_stream_t stream) {
+  if (!x || !xa || B < 1 || D < 1 || T < 1 || !dtype_ok(dtype)) return SFM_ERR_INVALID_ARG;
+  if (T + 2 > SFM_MAX_L) return SFM_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(xa)) return SFM_ERR_MISALIGNED;
+  const int es = esize_of(dtype);
+  if (overlaps(x, (long long)B * D * T * es, xa, (long long)B * D * (T + 2) * es)) return SFM_ERR_INVALID_ARG;
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_aux_init(x, xa, B, D, T, es, stream));
+}
+
+sfm_status sfm_aux_swap(void* y, int B, int D, int L, sfm_dtype dtype, sfm_stream_t stream) {
+  if (!y || B < 1 || D < 1 || L < 2 || !dtype_ok(dtype)) return SFM_ERR_INVALID_ARG;
+  if (L > SFM_MAX_L) return SFM_ERR_UNSUPPORTED;
+  if (!aligned16(y)) return SFM_ERR_MISALIGNED;
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_aux_swap(y, B, D, L, esize_of(dtype), stream));
+}
+
+sfm_status sfm_fold_conv1d(const void* x, const float* w, const float* bias, void* u, int B, int D, int L, int K,
+                           int pad_left, int B2, int silu, sfm_dtype dtype, sfm_stream_t stream) {
+  if (!x || !w || !u || B < 1 || D < 1 || L < 1 || !dtype_ok(dtype)) return SFM_ERR_INVALID_ARG;
+  if (K < 1 || K > SFM_MAX_K || pad_left < 0 || pad_left >= K) return SFM_ERR_INVALID_ARG;
+  if (B2 < 1 || B % B2 != 0 || (silu & ~1)) return SFM_ERR_INVALID_ARG;
+  if (L > SFM_MAX_L) return SFM_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(u)) return SFM_ERR_MISALIGNED;
+  const long long bytes = (long long)B * D * L * esize_of(dtype);
+  if (overlaps(x, bytes, u, bytes)) return SFM_ERR_INVALID_ARG;
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_conv1d(x, w, bias, u, B, D, L, K, pad_left, silu, dtype, stream));
+}
+
+sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* out) {
+  if (!out || B < 1 || T < 1 || D < 1 || N < 1) return SFM_ERR_INVALID_ARG;
+  *out = choose(B, T, D, N);
+  return SFM_OK;
+}
+
+sfm_status sfm_choose_b1(int B, int T, int D, int N, int* B1_out) {
+  if (!B1_out) return SFM_ERR_INVALID_ARG;
+  sfm_variant v;
+  sfm_status st = sfm_choose_variant(B, T, D, N, &v);
+  if (st != SFM_OK) return st;
+  *B1_out = v.B1;
+  return SFM_OK;
+}
+
+sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) {
+  sfm_status st = validate_scan(a, false);
+  if (st != SFM_OK) return st;
+  const int T = a->aux_init ? a->L - 2 : a->L;
+  const sfm_variant v = choose(a->B, T, a->D, a->N);
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.x = a->x;
+  p.dt = a->dt;
+  p.z = a->z;
+  p.Bm = a->Bm;
+  p.Cm = a->Cm;
+  p.A = a->A;
+  p.Dskip = a->Dskip;
+  p.dt_bias = a->dt_bias;
+  p.conv_w = a->conv_w;
+  p.conv_b = a->conv_b;
+  p.y = a->y;
+  p.final_state = a->final_state;
+  p.B = a->B;
+  p.D = a->D;
+  p.L = a->L;
+  p.N = a->N;
+  p.Tx = a->aux_init ? a->L - 2 : a->L;
+  p.K = a->conv_w ? a->K : 1;
+  p.pad_left = a->conv_w ? a->pad_left : 0;
+  p.B2 = a->B / (a->B1 ? a->B1 : v.B1);
+  p.d_tile = a->d_tile ? a->d_tile : v.d_tile;
+  p.chunk = a->chunk ? a->chunk : v.chunk;
+  p.flags = (a->dt_softplus ? kSoftplus : 0) | (a->aux_init ? kAuxInit : 0) |
+            (a->swap_out && a->L >= 2 ? kSwapOut : 0) | (a->conv_w ? kConv : 0) | (a->z ? kGate : 0);
+  const int si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);
+  int NP = 2;
+  while (NP < a->N) NP <<= 1;
+  if (a->B / p.B2 > kMaxB1) return SFM_ERR_UNSUPPORTED;
+  // whole-sample mode: the chunk covers the sample and every slab of every tensor starts
+  // on a 16-byte boundary with a size that is a multiple of 16 bytes (bulk-copy rules)
+  auto slab_ok = [&](long long per_row_bytes) {
+    const long long rem = (long long)(a->D % p.d_tile) * per_row_bytes;
+    return ((long long)a->D * per_row_bytes) % 16 == 0 && ((long long)p.d_tile * per_row_bytes) % 16 == 0 &&
+           rem % 16 == 0;
+  };
+  const bool aligned = slab_ok((long long)p.Tx * si) && slab_ok((long long)a->L * si) &&
+                       slab_ok((long long)a->L * so) && ((long long)a->N * a->L * si) % 16 == 0;
+  p.mode = kModeChunk;
+  if (p.chunk >= a->L && aligned) {
+    p.mode = kModeWhole;
+    p.smem_bytes = fwd_whole_smem(p, si, so, NP);
+    if (p.smem_bytes > kWholeSmemCap) p.mode = kModeChunk;
+  }
+  if (p.mode == kModeChunk) {
+    if (p.chunk > kMaxChunk) p.chunk = kMaxChunk;
+    p.x_row = fwd_x_row(p.chunk, 4, si);
+    p.io_row = fwd_io_row(p.chunk, si);
+    p.y_row = fwd_y_row(p.chunk, so);
+    p.smem_bytes = fwd_chunk_smem(p, si, so, NP);
+    if (p.smem_bytes > fwd_max_smem()) {
+      if (a->chunk || a->d_tile) return SFM_ERR_UNSUPPORTED;  // explicit shape that does not fit
+      while (p.smem_bytes > fwd_max_smem() && p.d_tile > 32) {
+        p.d_tile /= 2;
+        p.smem_bytes = fwd_chunk_smem(p, si, so, NP);
+      }
+      if (p.smem_bytes > fwd_max_smem()) return SFM_ERR_UNSUPPORTED;
+    }
+  }
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_fwd(p, a->in_dtype, a->out_dtype, NP, stream));
+}
+
+sfm_status sfm_scan_bwd_workspace_size(const sfm_scan_args* a, size_t* bytes) {
+  (void)a;
+  if (bytes) *bytes = 0;
+  return SFM_ERR_UNSUPPORTED;
+}
+
+sfm_status sfm_selective_scan_fold_bwd(const sfm_scan_args* a, const sfm_scan_grads* g, void* ws, size_t wsb,
+                                       sfm_stream_t stream) {
+  (void)a;
+  (void)g;
+  (void)ws;
+  (void)wsb;
+  (void)stream;
+  return SFM_ERR_UNSUPPORTED;
+}
+
+sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code) {
+  if (!code) return SFM_ERR_INVALID_ARG;
+  unsigned v = 0;
+  const sfm_status st = cuda_status(read_device_error(stream, clear, &v));
+  if (st != SFM_OK) return st;
+  *code = (int)v;
+  return SFM_OK;
+}
+
+}  // extern "C"

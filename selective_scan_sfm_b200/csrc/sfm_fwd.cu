@@ -1,0 +1,653 @@
+// sfm_fwd.cu -- fused forward of the SF-Mamba mixer hot path on B200 (sm_100a).
+//
+// One launch computes, for a tile of channels and one folded row of B2 samples:
+//   [aux init] -> depthwise conv (zero outside the sample) + SiLU -> Delta = softplus
+//   -> selective scan with the state restarted at every sample start -> D skip
+//   -> SiLU(z) gate -> [head<->tail swap] -> store.
+// Sources: "SF-Mamba: Scan Folding" (sungsoo.github.io) sections 3.1-3.3 and 8.1;
+// "SF-Mamba: Rethinking Vision Mamba" (techloop.online), Auxiliary Patch Swapping and
+// Batch Folding with Periodic State Reset.
+//
+// Schedule.  Grid = (channel tiles, B1 folded rows).  Each thread owns one channel and
+// walks the folded row p = 0 .. B2*L-1 in order with its N fp32 states in registers
+// (packed in pairs for the f32x2 FMA pipe).  The reset at p mod L == 0 makes the
+// transition factor of every sample's first token 0: the state restarts there and no
+// exp is evaluated.  The work is bound by the transcendental unit (N exp2 per token),
+// so the inner loop is built to keep it fed: interior tokens are processed in unrolled
+// groups with branch-free conv windows, so that one token's exps overlap the previous
+// token's state updates; tokens whose conv window touches an aux token or the
+// sample's zero padding (at most K per sample) take a general path.
+//
+// Staging, two modes:
+//  * whole-sample: when a sample's rows fit in shared memory and every slab is 16-byte
+//    aligned, the CTA's slab of each tensor -- [b, d0:d0+Dt, :], contiguous in memory --
+//    arrives with ONE bulk asynchronous copy (the TMA engine, no multicast) completing
+//    on an mbarrier, and the output slab leaves with one bulk store.
+//  * chunked: tokens are staged in chunks; each row segment is copied with 16-byte
+//    cp.async granules starting at the granule that holds its first element (rows of
+//    odd length are never 16-byte aligned, which rules out tensor maps and per-row bulk
+//    copies), and each thread reads its row at that row's byte offset.
+// B and C of the staged tokens are transposed once per CTA into fp32 [token][2N] so a
+// thread reads the N values of a token as 128-bit broadcast loads.
+#include <type_traits>
+
+#include "sfm_device.cuh"
+#include "sfm_internal.h"
+
+namespace sfm {
+
+__device__ unsigned int g_device_error = 0;
+
+constexpr int kGroup = 4;                      // tokens per unrolled group
+constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded wait on a bulk copy: 2 s
+
+__host__ __device__ inline int round16(int v) { return (v + 15) & ~15; }
+
+// Row stride (bytes) of a staged row of `cnt` elements (chunked mode): room for the
+// up-to-15 head bytes of the granule copy, and an odd number of 16-byte units.
+__host__ __device__ inline int stage_row_bytes(int cnt, int esize) {
+  int b = round16(cnt * esize + 15);
+  if (((b >> 4) & 1) == 0) b += 16;
+  return b;
+}
+
+// Output row stride when the output cannot overwrite the dt row in place (chunked mode).
+__host__ __device__ inline int out_row_bytes(int cnt, int esize) {
+  int b = (cnt * esize + 3) & ~3;
+  if (((b >> 2) & 1) == 0) b += 4;
+  return b;
+}
+
+// ------------------------------------------------------------------ mbarrier + bulk copy
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Polls the barrier until the phase with `parity` completes or kWaitNs elapse.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kWaitNs) return false;
+  return true;
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void bulk_s2g(void* dst, const void* src, unsigned bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;\n" ::"l"(dst), "r"(smem_u32(src)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;\n" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
+
+// ------------------------------------------------------------------ per-token arithmetic
+
+// Per-channel constants and state.  NH = pairs of states (N padded to an even count;
+// padded states have A = B = C = 0 and stay 0).
+template <int NH>
+struct Chan {
+  float2 h[NH];
+  float2 A2[NH];  // A * log2(e)
+  float w[4];
+  float cb, dsk, dtb, mean;
+};
+
+// State update and read-out of one token:
+//   h = Abar*h + Delta*B*u (Abar = 0 on a reset token), returns sum_n C_n h_n.
+template <int NH, bool RESET>
+__device__ __forceinline__ float scan_token(Chan<NH>& c, const float* __restrict__ bc, float delta, float dbu) {
+  const float2 d2 = make_float2(delta, delta), u2 = make_float2(dbu, dbu);
+  float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < NH; k += (NH % 2 == 0 ? 2 : 1)) {
+    float2 Bp[2], Cp[2];
+    if constexpr (NH % 2 == 0) {
+      const float4 b4 = *reinterpret_cast<const float4*>(bc + 2 * k);
+      const float4 c4 = *reinterpret_cast<const float4*>(bc + 2 * NH + 2 * k);
+      Bp[0] = make_float2(b4.x, b4.y);
+      Bp[1] = make_float2(b4.z, b4.w);
+      Cp[0] = make_float2(c4.x, c4.y);
+      Cp[1] = make_float2(c4.z, c4.w);
+    } else {
+      Bp[0] = *reinterpret_cast<const float2*>(bc + 2 * k);
+      Cp[0] = *reinterpret_cast<const float2*>(bc + 2 * NH + 2 * k);
+    }
+#pragma unroll
+    for (int j = 0; j < (NH % 2 == 0 ? 2 : 1); ++j) {
+      const float2 bu = __fmul2_rn(Bp[j], u2);
+      if constexpr (RESET) {
+        c.h[k + j] = bu;
+      } else {
+        float2 a = __fmul2_rn(d2, c.A2[k + j]);
+        a.x = ex2(a.x);
+        a.y = ex2(a.y);
+        c.h[k + j] = __ffma2_rn(a, c.h[k + j], bu);
+      }
+      if (j == 0)
+        ya = __ffma2_rn(Cp[j], c.h[k + j], ya);
+      else
+        yb = __ffma2_rn(Cp[j], c.h[k + j], yb);
+    }
+  }
+  const float2 s = __fadd2_rn(ya, yb);
+  return s.x + s.y;
+}
+
+// Runtime options of the general path.
+struct Opts {
+  int L, K, pl, off, Tx;  // off = 1 with aux tokens
+  bool conv, gate, sp, aux;
+};
+
+// Output of one token from its conv taps (xw[0..3] = xa[t-pl .. t-pl+3]), raw dt and z.
+// STD: conv (K = 4) + softplus + gate, all compile-time; else the runtime options.
+template <typename TI, int NH, bool STD, bool RESET>
+__device__ __forceinline__ float token_out(Chan<NH>& c, const Opts& o, const float* xw, TI dtv, TI zv,
+                                           const float* __restrict__ bc) {
+  float u;
+  if (STD || o.conv) {
+    float acc = c.cb;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (STD || q < o.K) acc = fmaf(c.w[q], xw[q], acc);
+    u = silu(acc);
+  } else {
+    u = xw[0];
+  }
+  const float v = to_f(dtv) + c.dtb;
+  const float delta = (STD || o.sp) ? softplus(v) : v;
+  float yv = scan_token<NH, RESET>(c, bc, delta, delta * u);
+  yv = fmaf(c.dsk, u, yv);
+  if (STD || o.gate) yv *= silu(to_f(zv));
+  return yv;
+}
+
+// xa at position s of the sample from the x row `xr` (x index q at xr[q - xlo]); aux
+// tokens are the mean; zero outside the sample or outside the staged window.
+template <typename TI>
+__device__ __forceinline__ float xa_at(const Opts& o, const TI* xr, int xlo, int xhi, float mean, int s) {
+  if (s < 0 || s >= o.L) return 0.0f;
+  if (o.aux) {
+    if (s == 0 || s == o.L - 1) return mean;
+    s -= 1;
+  }
+  if (s < xlo || s >= xhi) return 0.0f;
+  return to_f(xr[s - xlo]);
+}
+
+// General path for token t (chunk-relative i): conv taps with explicit boundary handling.
+template <typename TI, typename TO, int NH, bool STD>
+__device__ __forceinline__ float general_token(Chan<NH>& c, const Opts& o, const TI* xr, int xlo, int xhi, int t,
+                                               TI dtv, TI zv, const float* bc) {
+  float xw[4];
+  const int K = (STD || o.conv) ? 4 : 1, pl = (STD || o.conv) ? o.pl : 0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) xw[q] = q < K ? xa_at<TI>(o, xr, xlo, xhi, c.mean, t - pl + q) : 0.0f;
+  if (t == 0) return token_out<TI, NH, STD, true>(c, o, xw, dtv, zv, bc);
+  return token_out<TI, NH, STD, false>(c, o, xw, dtv, zv, bc);
+}
+
+// G interior tokens starting at chunk-relative index i: loads first (x window, dt, z),
+// then the G token computations, then the stores, so the compiler can overlap tokens.
+// xb[i + q] is the conv tap q of token i (no boundary inside the group).
+template <typename TI, typename TO, int NH, bool STD, int G>
+__device__ __forceinline__ void fast_group(Chan<NH>& c, const Opts& o, const TI* __restrict__ xb,
+                                           const TI* dtr, const TI* zr, TO* yr, int i,
+                                           const float* __restrict__ bct) {
+  constexpr int NP2 = 4 * NH;  // floats per token in bct
+  float xv[G + 3];
+#pragma unroll
+  for (int q = 0; q < G + 3; ++q) xv[q] = (q < G || STD || o.conv) ? to_f(xb[i + q]) : 0.0f;
+  TI dv[G], zv[G];
+#pragma unroll
+  for (int k = 0; k < G; ++k) {
+    dv[k] = dtr[i + k];
+    zv[k] = (STD || o.gate) ? zr[i + k] : dv[k];
+  }
+  float yv[G];
+#pragma unroll
+  for (int k = 0; k < G; ++k) yv[k] = token_out<TI, NH, STD, false>(c, o, xv + k, dv[k], zv[k], bct + (i + k) * NP2);
+#pragma unroll
+  for (int k = 0; k < G; ++k) yr[i + k] = from_f<TO>(yv[k]);
+}
+
+// Walks tokens [t0, t0 + cnt) of one sample.  xr: x row holding x indices [xlo, xhi);
+// dtr/zr/yr: rows indexed chunk-relative; bct: transposed B/C of the chunk.
+template <typename TI, typename TO, int NH, bool STD>
+__device__ __forceinline__ void walk(Chan<NH>& c, const Opts& o, const TI* xr, int xlo, int xhi, const TI* dtr,
+                                     const TI* zr, TO* yr, const float* bct, int t0, int cnt) {
+  constexpr int NP2 = 4 * NH;
+  // interior tokens: every conv tap on a plain x token; never the reset token
+  int ta = 1, tb = 0;
+  if (STD) {
+    ta = max(o.off + o.pl, 1);
+    tb = o.off + o.Tx - 4 + o.pl + 1;
+  }
+  const int tend = t0 + cnt;
+  const int e1 = min(tend, max(t0, ta));
+  const int e2 = max(e1, min(tend, tb));
+  for (int t = t0; t < e1; ++t) {
+    const int i = t - t0;
+    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
+  }
+  if (e2 > e1) {
+    // x index of tap 0 of token t is t - pl - off; xb[i + q] must be that + q
+    const TI* xb = xr + (t0 - o.pl - o.off - xlo);
+    int i = e1 - t0;
+    const int iend = e2 - t0;
+    for (; i + kGroup <= iend; i += kGroup) fast_group<TI, TO, NH, STD, kGroup>(c, o, xb, dtr, zr, yr, i, bct);
+    for (; i < iend; ++i) fast_group<TI, TO, NH, STD, 1>(c, o, xb, dtr, zr, yr, i, bct);
+  }
+  for (int t = e2; t < tend; ++t) {
+    const int i = t - t0;
+    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
+  }
+}
+
+template <int NH>
+__device__ __forceinline__ void load_chan(Chan<NH>& c, const FwdParams& p, int d, bool conv) {
+  const int N = p.N;
+#pragma unroll
+  for (int k = 0; k < NH; ++k) {
+    const int n0 = 2 * k, n1 = 2 * k + 1;
+    c.A2[k] = make_float2(n0 < N ? p.A[(size_t)d * N + n0] * kLog2e : 0.f,
+                          n1 < N ? p.A[(size_t)d * N + n1] * kLog2e : 0.f);
+    c.h[k] = make_float2(0.f, 0.f);
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) c.w[q] = (conv && q < p.K) ? p.conv_w[(size_t)d * p.K + q] : 0.0f;
+  c.cb = (conv && p.conv_b) ? p.conv_b[d] : 0.0f;
+  c.dsk = p.Dskip ? p.Dskip[d] : 0.0f;
+  c.dtb = p.dt_bias ? p.dt_bias[d] : 0.0f;
+  c.mean = 0.0f;
+}
+
+// B, C [N][cnt] (raw, element (n,i) at src + head_n + i*si) -> fp32 [cnt][4*NH] (B pairs
+// then C pairs), zero for padded states.
+template <typename TI, int NH>
+__device__ __forceinline__ void transpose_bc(float* bct, const char* bs, const char* cs, int row_bytes,
+                                             unsigned e0_base, unsigned L, int N, int cnt, int tid, int nthr,
+                                             bool per_row_head) {
+  constexpr int NP = 2 * NH, si = sizeof(TI);
+  for (int e = tid; e < cnt * NP; e += nthr) {
+    const int i = e / NP, n = e % NP;
+    float bv = 0.0f, cv = 0.0f;
+    if (n < N) {
+      // only the low 4 bits of the byte offset matter: 32-bit arithmetic is exact there
+      const int hb = per_row_head ? (int)(((e0_base + (unsigned)n * L) * si) & 15u) : 0;
+      const int off = n * row_bytes + hb + i * si;
+      bv = to_f(*reinterpret_cast<const TI*>(bs + off));
+      cv = to_f(*reinterpret_cast<const TI*>(cs + off));
+    }
+    bct[i * 2 * NP + n] = bv;
+    bct[i * 2 * NP + NP + n] = cv;
+  }
+}
+
+template <typename TI>
+__device__ __forceinline__ float row_mean(const TI* xr, int Tx) {
+  float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+  int t = 0;
+  for (; t + 4 <= Tx; t += 4) {
+    s0 += to_f(xr[t]);
+    s1 += to_f(xr[t + 1]);
+    s2 += to_f(xr[t + 2]);
+    s3 += to_f(xr[t + 3]);
+  }
+  for (; t < Tx; ++t) s0 += to_f(xr[t]);
+  return ((s0 + s1) + (s2 + s3)) / (float)Tx;
+}
+
+__device__ __forceinline__ Opts make_opts(const FwdParams& p) {
+  Opts o;
+  o.L = p.L;
+  o.conv = p.flags & kConv;
+  o.gate = p.flags & kGate;
+  o.sp = p.flags & kSoftplus;
+  o.aux = p.flags & kAuxInit;
+  o.K = o.conv ? p.K : 1;
+  o.pl = o.conv ? p.pad_left : 0;
+  o.off = o.aux ? 1 : 0;
+  o.Tx = p.Tx;
+  return o;
+}
+
+// ------------------------------------------------------------------ whole-sample mode
+
+// Shared memory: [barrier 16 B][x slab][dt slab][z slab][B][C][bct][y slab if not in place]
+template <typename TI, typename TO, int NH, bool STD>
+__global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
+  constexpr bool kInPlace = std::is_same<TI, TO>::value;
+  constexpr int si = sizeof(TI), so = sizeof(TO), NP = 2 * NH;
+  extern __shared__ __align__(16) char smem[];
+
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int d0 = blockIdx.x * p.d_tile;
+  const int dcount = min(p.d_tile, p.D - d0);
+  const int b1 = blockIdx.y;
+  const bool active = tid < dcount;
+  const int d = d0 + (active ? tid : 0);
+  const int L = p.L, N = p.N, Tx = p.Tx;
+  const Opts o = make_opts(p);
+  const bool swap = p.flags & kSwapOut;
+
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem);
+  volatile int& abort_flag = *reinterpret_cast<int*>(smem + 8);
+  char* xs = smem + 16;
+  char* dts = xs + round16(p.d_tile * Tx * si);
+  char* zs = dts + round16(p.d_tile * L * si);
+  char* bs = zs + (o.gate ? round16(p.d_tile * L * si) : 0);
+  char* cs = bs + round16(N * L * si);
+  float* bct = reinterpret_cast<float*>(cs + round16(N * L * si));
+  char* ys = reinterpret_cast<char*>(bct + L * 2 * NP);
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+
+  Chan<NH> c;
+  load_chan(c, p, d, o.conv);
+
+  const unsigned xbytes = (unsigned)(dcount * Tx * si), iobytes = (unsigned)(dcount * L * si);
+  const unsigned bcbytes = (unsigned)(N * L * si), ybytes = (unsigned)(dcount * L * so);
+  const char* xg = static_cast<const char*>(p.x);
+  const char* dtg = static_cast<const char*>(p.dt);
+  const char* zg = static_cast<const char*>(p.z);
+  const char* bg = static_cast<const char*>(p.Bm);
+  const char* cg = static_cast<const char*>(p.Cm);
+  char* yg = static_cast<char*>(p.y);
+
+  for (int j = 0; j < p.B2; ++j) {
+    const int b = b1 * p.B2 + j;
+    const long long row0 = (long long)b * p.D + d0;
+    if (tid == 0) {
+      if (j > 0) bulk_wait_read0();  // the previous output slab has been read out of smem
+      fence_proxy_async();
+      mbar_expect_tx(bar, xbytes + iobytes * (o.gate ? 2u : 1u) + 2u * bcbytes);
+      bulk_g2s(xs, xg + row0 * Tx * si, xbytes, bar);
+      bulk_g2s(dts, dtg + row0 * L * si, iobytes, bar);
+      if (o.gate) bulk_g2s(zs, zg + row0 * L * si, iobytes, bar);
+      bulk_g2s(bs, bg + (long long)b * N * L * si, bcbytes, bar);
+      bulk_g2s(cs, cg + (long long)b * N * L * si, bcbytes, bar);
+      if (!mbar_wait_bounded(bar, j & 1)) {
+        atomicExch(&g_device_error, (unsigned)SFM_ERR_TIMEOUT);
+        mbar_wait_bounded(bar, j & 1);  // give the copies in flight one more bounded chance
+        abort_flag = 1;
+      }
+    }
+    __syncthreads();
+    if (abort_flag) {
+      if (tid == 0) bulk_wait0();
+      return;
+    }
+    mbar_try_wait(bar, j & 1);  // completed: acquire the copied bytes in every thread
+
+    transpose_bc<TI, NH>(bct, bs, cs, L * si, 0u, (unsigned)L, N, L, tid, nthr, false);
+    if (active && o.aux) c.mean = row_mean(reinterpret_cast<const TI*>(xs) + tid * Tx, Tx);
+    __syncthreads();
+
+    if (active) {
+      const TI* xr = reinterpret_cast<const TI*>(xs) + tid * Tx;
+      const TI* dtr = reinterpret_cast<const TI*>(dts) + tid * L;
+      const TI* zr = o.gate ? reinterpret_cast<const TI*>(zs) + tid * L : dtr;
+      TO* yr = kInPlace ? reinterpret_cast<TO*>(dts) + tid * L : reinterpret_cast<TO*>(ys) + tid * L;
+#pragma unroll
+      for (int k = 0; k < NH; ++k) c.h[k] = make_float2(0.f, 0.f);
+      walk<TI, TO, NH, STD>(c, o, xr, 0, Tx, dtr, zr, yr, bct, 0, L);
+      if (swap) {
+        const TO h0 = yr[0];
+        yr[0] = yr[L - 1];
+        yr[L - 1] = h0;
+      }
+      if (p.final_state) {
+        float* fs = p.final_state + ((size_t)b * p.D + d) * N;
+#pragma unroll
+        for (int k = 0; k < NH; ++k) {
+          if (2 * k < N) fs[2 * k] = c.h[k].x;
+          if (2 * k + 1 < N) fs[2 * k + 1] = c.h[k].y;
+        }
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {
+      fence_proxy_async();  // the threads' smem writes become visible to the bulk store
+      bulk_s2g(yg + row0 * L * so, kInPlace ? dts : ys, ybytes);
+      bulk_commit();
+    }
+  }
+  if (tid == 0) bulk_wait0();
+}
+
+// ------------------------------------------------------------------ chunked mode
+
+template <typename TI, typename TO, int NH, bool STD>
+__global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
+  constexpr bool kInPlace = std::is_same<TI, TO>::value;
+  constexpr int si = sizeof(TI), so = sizeof(TO), NP = 2 * NH;
+  extern __shared__ __align__(16) char smem[];
+
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+  const int d0 = blockIdx.x * p.d_tile;
+  const int dcount = min(p.d_tile, p.D - d0);
+  const int b1 = blockIdx.y;
+  const bool active = tid < dcount;
+  const int d = d0 + (active ? tid : 0);
+  const int L = p.L, N = p.N, S = p.chunk, Tx = p.Tx;
+  const Opts o = make_opts(p);
+  const bool swap = p.flags & kSwapOut;
+  const int K = o.conv ? o.K : 1, pl = o.pl;
+
+  char* xs = smem;
+  char* dts = xs + p.d_tile * p.x_row;
+  char* zs = dts + p.d_tile * p.io_row;
+  char* bs = zs + (o.gate ? p.d_tile * p.io_row : 0);
+  char* cs = bs + N * p.io_row;
+  float* bct = reinterpret_cast<float*>(cs + N * p.io_row);
+  char* ys = reinterpret_cast<char*>(bct + S * 2 * NP);
+
+  Chan<NH> c;
+  load_chan(c, p, d, o.conv);
+
+  const long long x_bytes = (long long)p.B * p.D * Tx * si;
+  const long long io_bytes = (long long)p.B * p.D * L * si;
+  const long long bc_bytes = (long long)p.B * N * L * si;
+  const char* xg = static_cast<const char*>(p.x);
+  const char* dtg = static_cast<const char*>(p.dt);
+  const char* zg = static_cast<const char*>(p.z);
+  const char* bg = static_cast<const char*>(p.Bm);
+  const char* cg = static_cast<const char*>(p.Cm);
+  TO* yg = static_cast<TO*>(p.y);
+  const int nchunks = (L + S - 1) / S;
+
+  for (int j = 0; j < p.B2; ++j) {
+    const int b = b1 * p.B2 + j;
+    const long long row0 = (long long)b * p.D + d0;
+    const long long myrow = row0 + tid;
+    c.mean = (o.aux && active) ? row_mean(reinterpret_cast<const TI*>(xg) + myrow * Tx, Tx) : 0.0f;
+#pragma unroll
+    for (int k = 0; k < NH; ++k) c.h[k] = make_float2(0.f, 0.f);
+    TO head_val = from_f<TO>(0.0f);
+
+    for (int kc = 0; kc < nchunks; ++kc) {
+      const int t0 = kc * S, cnt = min(S, L - t0);
+      int slo = t0 - pl - o.off, shi = t0 + cnt - 1 + (K - 1 - pl) - o.off;
+      const int xlo = max(slo, 0), xhi = min(shi + 1, Tx);
+
+      // ---- stage: each thread copies its own rows; threads 0..2N-1 copy B and C rows
+      if (active) {
+        copy_span_async(xs + tid * p.x_row, xg, myrow * Tx + xlo, xhi - xlo, si, x_bytes, 0, 1);
+        copy_span_async(dts + tid * p.io_row, dtg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
+        if (o.gate) copy_span_async(zs + tid * p.io_row, zg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
+      }
+      for (int r = tid; r < 2 * N; r += nthr) {
+        const int n = r % N;
+        const long long e0 = ((long long)b * N + n) * L + t0;
+        copy_span_async((r < N ? bs : cs) + n * p.io_row, r < N ? bg : cg, e0, cnt, si, bc_bytes, 0, 1);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      __syncthreads();
+
+      transpose_bc<TI, NH>(bct, bs, cs, p.io_row, (unsigned)((long long)b * N * L + t0), (unsigned)L, N, cnt, tid,
+                           nthr, true);
+      __syncthreads();
+
+      if (active) {
+        const TI* xr = reinterpret_cast<const TI*>(xs + tid * p.x_row + span_head(myrow * Tx + xlo, si));
+        const int hd = span_head(myrow * L + t0, si);
+        const TI* dtr = reinterpret_cast<const TI*>(dts + tid * p.io_row + hd);
+        const TI* zr = o.gate ? reinterpret_cast<const TI*>(zs + tid * p.io_row + hd) : dtr;
+        TO* yr = kInPlace ? reinterpret_cast<TO*>(dts + tid * p.io_row + hd) : reinterpret_cast<TO*>(ys + tid * p.y_row);
+        walk<TI, TO, NH, STD>(c, o, xr, xlo, xhi, dtr, zr, yr, bct, t0, cnt);
+        if (swap) {
+          if (t0 == 0) head_val = yr[0];  // goes to position L-1
+          if (t0 + cnt == L) {
+            yg[myrow * L] = yr[cnt - 1];  // the tail output becomes the next head
+            yr[cnt - 1] = head_val;
+          }
+        }
+      }
+      __syncthreads();
+
+      // ---- store the chunk's outputs, coalesced along rows
+      for (int r = warp; r < dcount; r += nwarps) {
+        const long long rr = row0 + r;
+        const char* src = kInPlace ? dts + r * p.io_row + span_head(rr * L + t0, si) : ys + r * p.y_row;
+        TO* dst = yg + rr * L + t0;
+        for (int i = lane; i < cnt; i += 32)
+          if (!(swap && t0 + i == 0)) dst[i] = *reinterpret_cast<const TO*>(src + i * so);
+      }
+      // the next chunk's copies overwrite the staged rows only after every thread has
+      // passed the __syncthreads that follows them, i.e. after this loop
+    }
+
+    if (p.final_state && active) {
+      float* fs = p.final_state + ((size_t)b * p.D + d) * N;
+#pragma unroll
+      for (int k = 0; k < NH; ++k) {
+        if (2 * k < N) fs[2 * k] = c.h[k].x;
+        if (2 * k + 1 < N) fs[2 * k + 1] = c.h[k].y;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+int fwd_whole_smem(const FwdParams& p, int si, int so, int NP) {
+  const bool gate = p.flags & kGate;
+  long long s = 16;
+  s += round16(p.d_tile * p.Tx * si);
+  s += (long long)round16(p.d_tile * p.L * si) * (gate ? 2 : 1);
+  s += 2LL * round16(p.N * p.L * si);
+  s += (long long)p.L * 2 * NP * 4;
+  if (si != so) s += round16(p.d_tile * p.L * so);
+  return s > (1LL << 30) ? (1 << 30) : (int)s;
+}
+
+int fwd_chunk_smem(const FwdParams& p, int si, int so, int NP) {
+  const bool gate = p.flags & kGate;
+  long long s = 0;
+  s += (long long)p.d_tile * p.x_row;
+  s += (long long)p.d_tile * p.io_row * (gate ? 2 : 1);
+  s += 2LL * p.N * p.io_row;
+  s += (long long)p.chunk * 2 * NP * 4;
+  if (si != so) s += (long long)p.d_tile * p.y_row;
+  return s > (1LL << 30) ? (1 << 30) : (int)s;
+}
+
+int fwd_max_smem() { return 227 * 1024; }
+
+int fwd_x_row(int chunk, int K, int esize) { return stage_row_bytes(chunk + K - 1 + 1, esize); }
+int fwd_io_row(int chunk, int esize) { return stage_row_bytes(chunk, esize); }
+int fwd_y_row(int chunk, int esize) { return out_row_bytes(chunk, esize); }
+
+// Raises the kernel's dynamic shared-memory limit to `bytes` when it is not yet that high.
+// `have` caches the limit already set (a race only repeats the same call).
+template <typename Kern>
+static cudaError_t set_smem(Kern k, int bytes, int& have) {
+  if (bytes <= have) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
+
+template <typename TI, typename TO, int NH, bool STD>
+static cudaError_t launch_t(const FwdParams& p, cudaStream_t s) {
+  static int whole_set = 48 * 1024, chunk_set = 48 * 1024;
+  const int threads = (p.d_tile + 31) & ~31;
+  dim3 grid((p.D + p.d_tile - 1) / p.d_tile, p.B / p.B2);
+  cudaError_t e;
+  if (p.mode == kModeWhole) {
+    if ((e = set_smem(fwd_whole_kernel<TI, TO, NH, STD>, p.smem_bytes, whole_set)) != cudaSuccess) return e;
+    fwd_whole_kernel<TI, TO, NH, STD><<<grid, threads, p.smem_bytes, s>>>(p);
+  } else {
+    if ((e = set_smem(fwd_chunk_kernel<TI, TO, NH, STD>, p.smem_bytes, chunk_set)) != cudaSuccess) return e;
+    fwd_chunk_kernel<TI, TO, NH, STD><<<grid, threads, p.smem_bytes, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+template <typename TI, typename TO, int NH>
+static cudaError_t launch_std(const FwdParams& p, cudaStream_t s) {
+  const bool std_path = (p.flags & kConv) && (p.flags & kGate) && (p.flags & kSoftplus) && p.K == 4;
+  return std_path ? launch_t<TI, TO, NH, true>(p, s) : launch_t<TI, TO, NH, false>(p, s);
+}
+
+template <typename TI, typename TO>
+static cudaError_t launch_np(const FwdParams& p, int NP, cudaStream_t s) {
+  switch (NP) {
+    case 2: return launch_std<TI, TO, 1>(p, s);
+    case 4: return launch_std<TI, TO, 2>(p, s);
+    case 8: return launch_std<TI, TO, 4>(p, s);
+    case 16: return launch_std<TI, TO, 8>(p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fwd(const FwdParams& p, sfm_dtype in_dtype, sfm_dtype out_dtype, int NP, cudaStream_t s) {
+  if (in_dtype == SFM_F32 && out_dtype == SFM_F32) return launch_np<float, float>(p, NP, s);
+  if (in_dtype == SFM_BF16 && out_dtype == SFM_BF16) return launch_np<__nv_bfloat16, __nv_bfloat16>(p, NP, s);
+  if (in_dtype == SFM_BF16 && out_dtype == SFM_F32) return launch_np<__nv_bfloat16, float>(p, NP, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t read_device_error(cudaStream_t s, int clear, unsigned* value) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return e;
+  e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(unsigned));
+  if (e != cudaSuccess || !clear) return e;
+  const unsigned zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(unsigned));
+}
+
+}  // namespace sfm

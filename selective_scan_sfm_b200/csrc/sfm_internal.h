@@ -1,0 +1,63 @@
+// sfm_internal.h -- launch parameters shared by the host API and the kernels of libsfm.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+#include "sfm.h"
+
+namespace sfm {
+
+enum FwdFlags : int {
+  kSoftplus = 1 << 0,  // Delta = softplus(dt + dt_bias)
+  kAuxInit = 1 << 1,   // x holds T = L-2 tokens; aux tokens = mean, built on load
+  kSwapOut = 1 << 2,   // exchange output tokens 0 and L-1
+  kConv = 1 << 3,      // depthwise conv + SiLU on the input
+  kGate = 1 << 4,      // multiply by SiLU(z)
+};
+
+struct FwdParams {
+  const void* x;
+  const void* dt;
+  const void* z;
+  const void* Bm;
+  const void* Cm;
+  const float* A;
+  const float* Dskip;
+  const float* dt_bias;
+  const float* conv_w;
+  const float* conv_b;
+  void* y;
+  float* final_state;
+  int B, D, L, N, Tx;  // Tx = tokens per row of x (L-2 with aux init, else L)
+  int K, pad_left;
+  int B2;              // samples walked by one CTA (samples per folded row)
+  int d_tile;          // channels per CTA (= threads per CTA for one lane per channel)
+  int chunk;           // tokens staged per step of the walk
+  int flags;
+  int mode;            // kModeWhole or kModeChunk
+  // shared-memory carve-up (bytes), computed on the host
+  int x_row, io_row, y_row, smem_bytes;
+};
+
+// Staging modes of the forward kernel: whole-sample slabs by bulk copy, or token chunks.
+constexpr int kModeChunk = 0;
+constexpr int kModeWhole = 1;
+
+// Launchers (defined in the .cu files).  They only enqueue work; they return the
+// cudaError_t of the launch.
+cudaError_t launch_fwd(const FwdParams& p, sfm_dtype in_dtype, sfm_dtype out_dtype, int NP, cudaStream_t s);
+int fwd_whole_smem(const FwdParams& p, int in_size, int out_size, int NP);
+int fwd_chunk_smem(const FwdParams& p, int in_size, int out_size, int NP);
+int fwd_max_smem();
+int fwd_x_row(int chunk, int K, int esize);
+int fwd_io_row(int chunk, int esize);
+int fwd_y_row(int chunk, int esize);
+cudaError_t read_device_error(cudaStream_t s, int clear, unsigned* value);
+
+cudaError_t launch_aux_init(const void* x, void* xa, int B, int D, int T, int esize, cudaStream_t s);
+cudaError_t launch_aux_swap(void* y, int B, int D, int L, int esize, cudaStream_t s);
+cudaError_t launch_conv1d(const void* x, const float* w, const float* bias, void* u, int B, int D, int L, int K,
+                          int pad_left, int silu, sfm_dtype dtype, cudaStream_t s);
+
+}  // namespace sfm
