@@ -13,9 +13,9 @@
  *
  * Passages this follows:
  *   - recurrence h_t = Abar_t h_{t-1} + Bbar_t x_t, y_t = C_t h_t:
- *     "SF-Mamba: Scan Folding" (sungsoo.github.io), section 3.1;
+ *     "Seeing Both Ways, Running One Way" (sungsoo.github.io), section 3.1;
  *   - aux head/tail tokens initialised to avg(X), swapped head<->tail between layers:
- *     same page, section 3.2 equations; "SF-Mamba: Rethinking Vision Mamba"
+ *     same page, section 3.2 equations; "SF-Mamba：重新思考视觉 Mamba 的信息流与并行效率"
  *     (techloop.online), Auxiliary Patch Swapping;
  *   - folding [B,D,T] -> [B1,D,B2*T], B = B1*B2, with Abar_t = 0 at every sample start:
  *     sungsoo.github.io section 3.3 equations; techloop.online, Batch Folding with

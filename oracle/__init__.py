@@ -11,9 +11,9 @@ mixer layer from the single steps in the order the pages give:
     -> Delta = softplus(dt + dt_bias) -> selective scan with D skip -> y * SiLU(z)
     -> head<->tail swap of the output for the next layer.
 
-Sources: "SF-Mamba: Rethinking Vision Mamba" (techloop.online), sections on
+Sources: "SF-Mamba：重新思考视觉 Mamba 的信息流与并行效率" (techloop.online), sections on
 Auxiliary Patch Swapping and Batch Folding with Periodic State Reset;
-"SF-Mamba: Scan Folding" (sungsoo.github.io), section 3.1-3.3 equations and
+"Seeing Both Ways, Running One Way" (sungsoo.github.io), section 3.1-3.3 equations and
 section 8.1 items 1-5.  Pins for every function live in tests/test_oracle_pins.py.
 """
 from __future__ import annotations

@@ -8,7 +8,7 @@
  * Every routine is the plain definition written out, one sample at a time, in the
  * order the pages describe the method:
  *   - selective SSM recurrence h_t = Abar_t h_{t-1} + Bbar_t x_t, y_t = C_t h_t
- *     ("SF-Mamba: Scan Folding", sungsoo.github.io, section 3.1, the recurrence);
+ *     ("Seeing Both Ways, Running One Way", sungsoo.github.io, section 3.1, the recurrence);
  *   - discretisation Abar = exp(Delta*A), Bbar = Delta*B, D skip, SiLU(z) gate and
  *     Delta = softplus(dt + dt_bias): the standard Mamba convention (Gu & Dao, cited
  *     as background source 4 on the same page); the pages do not spell it out;

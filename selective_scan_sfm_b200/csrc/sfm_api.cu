@@ -136,6 +136,70 @@ sfm_status validate_scan(const sfm_scan_args* a, bool bwd) {
   return SFM_OK;
 }
 
+constexpr int kBwdDTile = 64;
+
+// The backward takes a plain scan (input u, no conv, no aux tokens, no swap).
+sfm_status validate_bwd_args(const sfm_scan_args* a) {
+  const sfm_status st = validate_scan(a, true);
+  if (st != SFM_OK) return st;
+  if (a->conv_w || a->aux_init || a->swap_out) return SFM_ERR_UNSUPPORTED;
+  return SFM_OK;
+}
+
+sfm_status validate_grads(const sfm_scan_args* a, const sfm_scan_grads* g) {
+  if (!g || g->size != sizeof(sfm_scan_grads)) return SFM_ERR_INVALID_ARG;
+  if (!g->dout || !g->du || !g->ddt || !g->dA || !g->dB || !g->dC) return SFM_ERR_INVALID_ARG;
+  if (a->z && !g->dz) return SFM_ERR_INVALID_ARG;
+  if (!aligned16(g->dout)) return SFM_ERR_MISALIGNED;
+  const float* outs[] = {g->du, g->ddt, g->dz, g->dA, g->dDskip, g->ddt_bias, g->dB, g->dC};
+  for (const float* o : outs)
+    if (o && (reinterpret_cast<uintptr_t>(o) & 3u)) return SFM_ERR_MISALIGNED;
+  const long long si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);
+  const long long bdl = (long long)a->B * a->D * a->L, bnl = (long long)a->B * a->N * a->L;
+  const void* ins[] = {a->x, a->dt, a->z, a->Bm, a->Cm, g->dout, a->A, a->Dskip, a->dt_bias};
+  const long long insz[] = {bdl * si, bdl * si, bdl * si, bnl * si, bnl * si, bdl * so,
+                            (long long)a->D * a->N * 4, (long long)a->D * 4, (long long)a->D * 4};
+  const long long outsz[] = {bdl * 4, bdl * 4, bdl * 4, (long long)a->D * a->N * 4, (long long)a->D * 4,
+                             (long long)a->D * 4, bnl * 4, bnl * 4};
+  for (int i = 0; i < 8; ++i) {
+    for (int j = 0; j < 9; ++j)
+      if (overlaps(outs[i], outsz[i], ins[j], insz[j])) return SFM_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 8; ++j)
+      if (overlaps(outs[i], outsz[i], outs[j], outsz[j])) return SFM_ERR_INVALID_ARG;
+  }
+  return SFM_OK;
+}
+
+BwdParams make_bwd_params(const sfm_scan_args* a, const sfm_scan_grads* g) {
+  BwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.u = a->x;
+  p.dt = a->dt;
+  p.z = a->z;
+  p.Bm = a->Bm;
+  p.Cm = a->Cm;
+  p.dout = g->dout;
+  p.A = a->A;
+  p.Dskip = a->Dskip;
+  p.dt_bias = a->dt_bias;
+  p.du = g->du;
+  p.ddt = g->ddt;
+  p.dz = a->z ? g->dz : nullptr;
+  p.dA = g->dA;
+  p.dDskip = a->Dskip ? g->dDskip : nullptr;
+  p.ddt_bias = a->dt_bias ? g->ddt_bias : nullptr;
+  p.dB = g->dB;
+  p.dC = g->dC;
+  p.B = a->B;
+  p.D = a->D;
+  p.L = a->L;
+  p.N = a->N;
+  p.d_tile = kBwdDTile;
+  p.ntiles = (a->D + kBwdDTile - 1) / kBwdDTile;
+  p.softplus = a->dt_softplus;
+  return p;
+}
+
 }  // namespace
 
 extern "C" {
@@ -272,19 +336,25 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
 }
 
 sfm_status sfm_scan_bwd_workspace_size(const sfm_scan_args* a, size_t* bytes) {
-  (void)a;
-  if (bytes) *bytes = 0;
-  return SFM_ERR_UNSUPPORTED;
+  if (!bytes) return SFM_ERR_INVALID_ARG;
+  const sfm_status st = validate_bwd_args(a);
+  if (st != SFM_OK) return st;
+  *bytes = bwd_workspace_bytes(a->B, a->D, a->L, a->N, kBwdDTile);
+  return SFM_OK;
 }
 
 sfm_status sfm_selective_scan_fold_bwd(const sfm_scan_args* a, const sfm_scan_grads* g, void* ws, size_t wsb,
                                        sfm_stream_t stream) {
-  (void)a;
-  (void)g;
-  (void)ws;
-  (void)wsb;
-  (void)stream;
-  return SFM_ERR_UNSUPPORTED;
+  sfm_status st = validate_bwd_args(a);
+  if (st != SFM_OK) return st;
+  if ((st = validate_grads(a, g)) != SFM_OK) return st;
+  if (!ws) return SFM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return SFM_ERR_MISALIGNED;
+  if (wsb < bwd_workspace_bytes(a->B, a->D, a->L, a->N, kBwdDTile)) return SFM_ERR_INVALID_ARG;
+  if (fault_injected()) return SFM_ERR_CUDA;
+  BwdParams p = make_bwd_params(a, g);
+  bwd_carve(p, static_cast<char*>(ws));
+  return cuda_status(launch_bwd(p, a->in_dtype, a->out_dtype, stream));
 }
 
 sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code) {

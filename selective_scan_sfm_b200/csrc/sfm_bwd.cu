@@ -1,0 +1,225 @@
+// sfm_bwd.cu -- backward of the folded selective scan (from its input u to the gated
+// output), sm_100a.
+//
+// Per sample b, channel d and state n, the adjoint of the state obeys
+//   g_t = C_t * dy_t + Abar_(t+1) * g_(t+1)   (no carry past the sample's last token)
+// where dy_t = dout_t * SiLU(z_t).  At a sample start the transition factor is the
+// constant 0 (the reset of "Seeing Both Ways, Running One Way", sungsoo.github.io,
+// section 3.3), so no gradient crosses samples and none flows into A, Delta or the
+// previous state through that token.
+//
+// Schedule (built for exact, reproducible sums rather than speed):
+//   bwd_main_kernel: grid (channel tiles, B); one thread per channel loops over the N
+//     states.  Per state: a forward sweep stores h_t in the workspace, a reverse sweep
+//     accumulates du, dDelta and dA in the caller's fp32 outputs / registers and writes
+//     each channel's dB/dC contribution; the CTA then sums those over its channels in a
+//     fixed order into per-tile partials.
+//   bwd_reduce_bc_kernel: dB, dC = sum of the tile partials, in tile order.
+//   bwd_reduce_param_kernel: dA, dDskip, ddt_bias = sum over samples, in sample order.
+#include "sfm_device.cuh"
+#include "sfm_internal.h"
+
+namespace sfm {
+
+__device__ __forceinline__ float sigmoid(float v) { return rcp(1.0f + ex2(-v * kLog2e)); }
+
+template <typename TI, typename TD>
+__global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int tile = blockIdx.x, b = blockIdx.y;
+  const int d0 = tile * p.d_tile;
+  const int dcount = min(p.d_tile, p.D - d0);
+  const bool active = tid < dcount;
+  const int d = d0 + (active ? tid : 0);
+  const int L = p.L, N = p.N;
+  const bool gate = p.z != nullptr, use_sp = p.softplus;
+  const size_t row = ((size_t)b * p.D + d) * L;
+
+  const TI* u = static_cast<const TI*>(p.u) + row;
+  const TI* dt = static_cast<const TI*>(p.dt) + row;
+  const TI* z = gate ? static_cast<const TI*>(p.z) + row : nullptr;
+  const TD* dout = static_cast<const TD*>(p.dout) + row;
+  const TI* Bm = static_cast<const TI*>(p.Bm) + (size_t)b * N * L;
+  const TI* Cm = static_cast<const TI*>(p.Cm) + (size_t)b * N * L;
+  const float dsk = p.Dskip ? p.Dskip[d] : 0.0f;
+  const float dtb = p.dt_bias ? p.dt_bias[d] : 0.0f;
+  float* du = p.du + row;
+  float* ddt = p.ddt + row;  // holds dLoss/dDelta until the final pass
+  float* dz = gate ? p.dz + row : nullptr;  // holds the pre-gate output y until the final pass
+  float* hb = p.hbuf + row;
+  float* cB = p.cB + row;
+  float* cC = p.cC + row;
+
+  auto delta_at = [&](int t) {
+    const float v = to_f(dt[t]) + dtb;
+    return use_sp ? softplus(v) : v;
+  };
+  auto gy_at = [&](int t) { return gate ? to_f(dout[t]) * silu(to_f(z[t])) : to_f(dout[t]); };
+
+  float sum_dsk = 0.0f;
+  if (active) {
+    for (int t = 0; t < L; ++t) {
+      const float gy = gy_at(t), ut = to_f(u[t]);
+      du[t] = gy * dsk;
+      ddt[t] = 0.0f;
+      if (gate) dz[t] = dsk * ut;
+      sum_dsk = fmaf(gy, ut, sum_dsk);
+    }
+  }
+
+  for (int n = 0; n < N; ++n) {
+    if (active) {
+      const float an = p.A[(size_t)d * N + n];
+      const TI* Bn = Bm + (size_t)n * L;
+      const TI* Cn = Cm + (size_t)n * L;
+      // forward sweep: h_t (the reset token starts from 0)
+      float h = 0.0f;
+      for (int t = 0; t < L; ++t) {
+        const float delta = delta_at(t);
+        const float bu = delta * to_f(Bn[t]) * to_f(u[t]);
+        h = t == 0 ? bu : fmaf(ex2(delta * an * kLog2e), h, bu);
+        hb[t] = h;
+        if (gate) dz[t] = fmaf(to_f(Cn[t]), h, dz[t]);
+      }
+      // reverse sweep
+      float g = 0.0f, a_next = 0.0f, dA = 0.0f;
+      for (int t = L - 1; t >= 0; --t) {
+        const float delta = delta_at(t), gy = gy_at(t), ut = to_f(u[t]), Bv = to_f(Bn[t]);
+        g = fmaf(gy, to_f(Cn[t]), t + 1 < L ? a_next * g : 0.0f);
+        cC[t] = gy * hb[t];
+        cB[t] = g * delta * ut;
+        du[t] = fmaf(g * delta, Bv, du[t]);
+        float dd = g * Bv * ut;
+        float a_t = 0.0f;
+        if (t > 0) {
+          a_t = ex2(delta * an * kLog2e);
+          const float gha = g * hb[t - 1] * a_t;  // dLoss/dAbar_t * Abar_t
+          dd = fmaf(gha, an, dd);
+          dA = fmaf(gha, delta, dA);
+        }
+        ddt[t] += dd;
+        a_next = a_t;
+      }
+      p.partA[((size_t)b * p.D + d) * N + n] = dA;
+    }
+    __syncthreads();
+    // this tile's share of dB[b,n,:] and dC[b,n,:], summed over its channels in order
+    for (int t = tid; t < L; t += nthr) {
+      float sb = 0.0f, sc = 0.0f;
+      const size_t base = ((size_t)b * p.D + d0) * L + t;
+      for (int c = 0; c < dcount; ++c) {
+        sb += p.cB[base + (size_t)c * L];
+        sc += p.cC[base + (size_t)c * L];
+      }
+      const size_t o = (((size_t)b * p.ntiles + tile) * 2) * N * L + (size_t)n * L + t;
+      p.partBC[o] = sb;
+      p.partBC[o + (size_t)N * L] = sc;
+    }
+    __syncthreads();
+  }
+
+  if (active) {
+    float sum_bias = 0.0f;
+    for (int t = 0; t < L; ++t) {
+      const float v = to_f(dt[t]) + dtb;
+      const float ds = use_sp ? ddt[t] * (v > 20.0f ? 1.0f : sigmoid(v)) : ddt[t];
+      ddt[t] = ds;
+      sum_bias += ds;
+      if (gate) {
+        const float zt = to_f(z[t]), sg = sigmoid(zt);
+        dz[t] = to_f(dout[t]) * dz[t] * (sg * (1.0f + zt * (1.0f - sg)));
+      }
+    }
+    p.partD[(size_t)b * p.D + d] = sum_dsk;
+    p.partBias[(size_t)b * p.D + d] = sum_bias;
+  }
+}
+
+// dB[b,n,t] / dC[b,n,t]: sum over channel tiles in tile order.
+__global__ void bwd_reduce_bc_kernel(const BwdParams p) {
+  const size_t NL = (size_t)p.N * p.L;
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (size_t)p.B * NL) return;
+  const size_t b = i / NL, r = i % NL;
+  float sb = 0.0f, sc = 0.0f;
+  for (int k = 0; k < p.ntiles; ++k) {
+    const size_t o = ((b * p.ntiles + k) * 2) * NL + r;
+    sb += p.partBC[o];
+    sc += p.partBC[o + NL];
+  }
+  p.dB[i] = sb;
+  p.dC[i] = sc;
+}
+
+// dA[d,n], dDskip[d], ddt_bias[d]: sum over samples in sample order.
+__global__ void bwd_reduce_param_kernel(const BwdParams p) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t DN = (size_t)p.D * p.N;
+  if (i < DN) {
+    float s = 0.0f;
+    for (int b = 0; b < p.B; ++b) s += p.partA[(size_t)b * DN + i];
+    p.dA[i] = s;
+  }
+  if (i < (size_t)p.D) {
+    float s0 = 0.0f, s1 = 0.0f;
+    for (int b = 0; b < p.B; ++b) {
+      s0 += p.partD[(size_t)b * p.D + i];
+      s1 += p.partBias[(size_t)b * p.D + i];
+    }
+    if (p.dDskip) p.dDskip[i] = s0;
+    if (p.ddt_bias) p.ddt_bias[i] = s1;
+  }
+}
+
+// Workspace carve-up: each region starts on a 256-byte boundary.
+static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+size_t bwd_workspace_bytes(int B, int D, int L, int N, int d_tile) {
+  const size_t bdl = (size_t)B * D * L, ntiles = (size_t)((D + d_tile - 1) / d_tile);
+  size_t s = 0;
+  s += 3 * align256(bdl * 4);                           // hbuf, cB, cC
+  s += align256((size_t)B * ntiles * 2 * N * L * 4);    // partBC
+  s += align256((size_t)B * D * N * 4);                 // partA
+  s += 2 * align256((size_t)B * D * 4);                 // partD, partBias
+  return s;
+}
+
+void bwd_carve(BwdParams& p, char* ws) {
+  const size_t bdl = (size_t)p.B * p.D * p.L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    float* r = reinterpret_cast<float*>(ws + o);
+    o += align256(bytes);
+    return r;
+  };
+  p.hbuf = take(bdl * 4);
+  p.cB = take(bdl * 4);
+  p.cC = take(bdl * 4);
+  p.partBC = take((size_t)p.B * p.ntiles * 2 * p.N * p.L * 4);
+  p.partA = take((size_t)p.B * p.D * p.N * 4);
+  p.partD = take((size_t)p.B * p.D * 4);
+  p.partBias = take((size_t)p.B * p.D * 4);
+}
+
+template <typename TI, typename TD>
+static cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
+  const int threads = (p.d_tile + 31) & ~31;
+  bwd_main_kernel<TI, TD><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t nbc = (size_t)p.B * p.N * p.L;
+  bwd_reduce_bc_kernel<<<(unsigned)((nbc + 255) / 256), 256, 0, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t np = (size_t)p.D * p.N > (size_t)p.D ? (size_t)p.D * p.N : (size_t)p.D;
+  bwd_reduce_param_kernel<<<(unsigned)((np + 255) / 256), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dtype, cudaStream_t s) {
+  if (in_dtype == SFM_F32 && dout_dtype == SFM_F32) return launch_bwd_t<float, float>(p, s);
+  if (in_dtype == SFM_BF16 && dout_dtype == SFM_BF16) return launch_bwd_t<__nv_bfloat16, __nv_bfloat16>(p, s);
+  if (in_dtype == SFM_BF16 && dout_dtype == SFM_F32) return launch_bwd_t<__nv_bfloat16, float>(p, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace sfm

@@ -4,8 +4,8 @@
 //   [aux init] -> depthwise conv (zero outside the sample) + SiLU -> Delta = softplus
 //   -> selective scan with the state restarted at every sample start -> D skip
 //   -> SiLU(z) gate -> [head<->tail swap] -> store.
-// Sources: "SF-Mamba: Scan Folding" (sungsoo.github.io) sections 3.1-3.3 and 8.1;
-// "SF-Mamba: Rethinking Vision Mamba" (techloop.online), Auxiliary Patch Swapping and
+// Sources: "Seeing Both Ways, Running One Way" (sungsoo.github.io) sections 3.1-3.3 and 8.1;
+// "SF-Mamba：重新思考视觉 Mamba 的信息流与并行效率" (techloop.online), Auxiliary Patch Swapping and
 // Batch Folding with Periodic State Reset.
 //
 // Schedule.  Grid = (channel tiles, B1 folded rows).  Each thread owns one channel and

@@ -44,6 +44,23 @@ struct FwdParams {
 constexpr int kModeChunk = 0;
 constexpr int kModeWhole = 1;
 
+struct BwdParams {
+  const void* u;
+  const void* dt;
+  const void* z;
+  const void* Bm;
+  const void* Cm;
+  const void* dout;
+  const float* A;
+  const float* Dskip;
+  const float* dt_bias;
+  float *du, *ddt, *dz, *dA, *dDskip, *ddt_bias, *dB, *dC;
+  // workspace regions (carved by bwd_carve)
+  float *hbuf, *cB, *cC, *partBC, *partA, *partD, *partBias;
+  int B, D, L, N, d_tile, ntiles;
+  int softplus;
+};
+
 // Launchers (defined in the .cu files).  They only enqueue work; they return the
 // cudaError_t of the launch.
 cudaError_t launch_fwd(const FwdParams& p, sfm_dtype in_dtype, sfm_dtype out_dtype, int NP, cudaStream_t s);
@@ -54,6 +71,10 @@ int fwd_x_row(int chunk, int K, int esize);
 int fwd_io_row(int chunk, int esize);
 int fwd_y_row(int chunk, int esize);
 cudaError_t read_device_error(cudaStream_t s, int clear, unsigned* value);
+
+cudaError_t launch_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dtype, cudaStream_t s);
+size_t bwd_workspace_bytes(int B, int D, int L, int N, int d_tile);
+void bwd_carve(BwdParams& p, char* ws);
 
 cudaError_t launch_aux_init(const void* x, void* xa, int B, int D, int T, int esize, cudaStream_t s);
 cudaError_t launch_aux_swap(void* y, int B, int D, int L, int esize, cudaStream_t s);

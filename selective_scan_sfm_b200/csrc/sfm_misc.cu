@@ -3,9 +3,9 @@
 // run the steps separately and the unfused comparison; the fused forward kernel does
 // the same work inside its loads and stores.
 //
-// Sources: "SF-Mamba: Scan Folding" (sungsoo.github.io) section 3.2 (aux tokens,
+// Sources: "Seeing Both Ways, Running One Way" (sungsoo.github.io) section 3.2 (aux tokens,
 // head<->tail swap) and section 8.1 item 5 (conv that does not cross folded sample
-// boundaries); "SF-Mamba: Rethinking Vision Mamba" (techloop.online), Auxiliary Patch
+// boundaries); "SF-Mamba：重新思考视觉 Mamba 的信息流与并行效率" (techloop.online), Auxiliary Patch
 // Swapping and the convolution-boundary paragraph.
 #include "sfm_device.cuh"
 #include "sfm_internal.h"

@@ -146,3 +146,39 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         _abi.lib()
+
+
+def good_grads(**kw):
+    g = _abi.ScanGrads()
+    g.size = ctypes.sizeof(_abi.ScanGrads)
+    base = FAKE + (16 << 24)
+    for i, k in enumerate(("dout", "du", "ddt", "dz", "dA", "dDskip", "ddt_bias", "dB", "dC")):
+        setattr(g, k, base + (i << 24))
+    for k, v in kw.items():
+        setattr(g, k, v)
+    return g
+
+
+def bwd_args(**kw):
+    kw.setdefault("conv_w", None)
+    kw.setdefault("conv_b", None)
+    kw.setdefault("aux_init", 0)
+    return good_args(**kw)
+
+
+def test_backward_workspace_query_and_validation(L, inject):
+    need = ctypes.c_size_t(0)
+    assert L.sfm_scan_bwd_workspace_size(ctypes.byref(bwd_args()), ctypes.byref(need)) == _abi.SFM_OK
+    assert need.value >= 3 * 4 * 16 * 51 * 4
+    assert L.sfm_scan_bwd_workspace_size(ctypes.byref(good_args()), ctypes.byref(need)) == _abi.SFM_ERR_UNSUPPORTED
+    ws = FAKE + (40 << 24)
+    call = lambda a, g, w=ws, n=need.value: L.sfm_selective_scan_fold_bwd(ctypes.byref(a), ctypes.byref(g), w, n, None)
+    assert call(bwd_args(), good_grads()) == _abi.SFM_ERR_CUDA           # valid: reaches the launch path
+    assert call(bwd_args(), good_grads(), n=need.value - 1) == _abi.SFM_ERR_INVALID_ARG
+    assert call(bwd_args(), good_grads(), w=ws + 16) == _abi.SFM_ERR_MISALIGNED
+    assert call(bwd_args(), good_grads(), w=None) == _abi.SFM_ERR_INVALID_ARG
+    assert call(bwd_args(swap_out=1), good_grads()) == _abi.SFM_ERR_UNSUPPORTED
+    assert call(bwd_args(), good_grads(dz=None)) == _abi.SFM_ERR_INVALID_ARG  # z given, dz missing
+    assert call(bwd_args(), good_grads(du=FAKE + (1 << 24))) == _abi.SFM_ERR_INVALID_ARG  # du aliases dt
+    assert call(bwd_args(), good_grads(size=4)) == _abi.SFM_ERR_INVALID_ARG
+    assert call(bwd_args(), good_grads(dA=FAKE + (20 << 24) + 2)) == _abi.SFM_ERR_MISALIGNED

@@ -1,0 +1,100 @@
+"""GPU parity of the scan backward against the fp64 oracle's reverse sweep.
+
+Per-element gradients (du, ddt, dz, dB, dC) use the metric of tests/parity.py; the
+reduced parameter gradients (dA, dDskip, ddt_bias) use the norm-wise ||g-r||_inf/||r||_inf."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_scan_sfm_b200 import SfmError, sfm_selective_scan_fold_bwd, synth
+
+from parity import TOL, rel_err, to_cuda
+
+pytestmark = pytest.mark.gpu
+
+PER_ELEMENT = ("du", "ddt", "dz", "dB", "dC")
+REDUCED = ("dA", "dDskip", "ddt_bias")
+
+
+def normwise(g, r):
+    g, r = np.asarray(g, np.float64), np.asarray(r, np.float64)
+    return float(np.max(np.abs(g - r)) / max(np.max(np.abs(r)), 1e-300))
+
+
+def run_both(d, dout, samples=None):
+    dc = to_cuda(d)
+    g = sfm_selective_scan_fold_bwd(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], dout.cuda(), z=dc["z"],
+                                    Dskip=dc["Dskip"], dt_bias=dc["dt_bias"])
+    torch.cuda.synchronize()
+    f = lambda t: t.double().numpy()
+    ref = oracle.scan_bwd(f(d["x"]), f(d["dt"]), f(d["Bm"]), f(d["Cm"]), f(d["A"]), f(dout), f(d["Dskip"]),
+                          f(d["dt_bias"]), f(d["z"]))
+    return {k: v.double().cpu().numpy() for k, v in g.items()}, ref
+
+
+def check_grads(g, ref, tol_elem, tol_red):
+    errs = {}
+    for k in PER_ELEMENT:
+        errs[k] = rel_err(g[k], ref[k])
+    for k in REDUCED:
+        errs[k] = normwise(g[k], ref[k])
+    bad = {k: e for k, e in errs.items() if e > (tol_elem if k in PER_ELEMENT else tol_red)}
+    assert not bad, "gradient errors above bound: %s (all: %s)" % (bad, errs)
+    return errs
+
+
+def test_backward_small_fp32():
+    d = synth.make_inputs(B=3, D=70, T=40, N=8, dtype="f32", seed=31, aux=False, random_A=True)
+    dout = synth.make_dout(3, 70, 40, seed=31, dtype="f32")
+    g, ref = run_both(d, dout)
+    check_grads(g, ref, TOL["f32"], TOL["f32"])
+
+
+def test_backward_is_bitwise_reproducible():
+    d = synth.make_inputs(B=4, D=130, T=51, N=16, dtype="bf16", seed=32, aux=False)
+    dc = to_cuda(d)
+    dout = synth.make_dout(4, 130, 51, seed=32).cuda()
+    run = lambda: sfm_selective_scan_fold_bwd(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], dout, z=dc["z"],
+                                              Dskip=dc["Dskip"], dt_bias=dc["dt_bias"])
+    a, b = run(), run()
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_backward_sample_isolation():
+    d = synth.make_inputs(B=4, D=64, T=30, N=8, dtype="f32", seed=33, aux=False)
+    dc = to_cuda(d)
+    dout = synth.make_dout(4, 64, 30, seed=33, dtype="f32").cuda()
+    run = lambda o: sfm_selective_scan_fold_bwd(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], o, z=dc["z"],
+                                                Dskip=dc["Dskip"], dt_bias=dc["dt_bias"])
+    g0 = run(dout)
+    o2 = dout.clone()
+    o2[1] = float("nan")
+    g1 = run(o2)
+    keep = [0, 2, 3]
+    for k in PER_ELEMENT:
+        assert torch.equal(g1[k][keep], g0[k][keep]), k
+
+
+def test_backward_workspace_errors():
+    d = to_cuda(synth.make_inputs(B=2, D=32, T=20, N=4, dtype="f32", seed=34, aux=False))
+    dout = torch.randn(2, 32, 20, device="cuda")
+    args = (d["x"], d["dt"], d["Bm"], d["Cm"], d["A"], dout)
+    with pytest.raises(SfmError, match="INVALID"):
+        sfm_selective_scan_fold_bwd(*args, workspace=torch.empty(64, dtype=torch.uint8, device="cuda"))
+    big = torch.empty(1 << 22, dtype=torch.uint8, device="cuda")
+    with pytest.raises(SfmError, match="MISALIGNED"):
+        sfm_selective_scan_fold_bwd(*args, workspace=big[16:])
+
+
+def test_backward_chain_stage3_shape_bf16():
+    """The backward at the four-layer chain's shape (B=64, D=640, L=198, N=16, bf16 inputs),
+    every gradient against the fp64 oracle on the full tensors."""
+    w = synth.WORKLOADS["chain4_stage3"]
+    d = synth.make_inputs(B=w["B"], D=w["D"], T=w["T"] + 2, N=w["N"], dtype="bf16", seed=4000, aux=False)
+    dout = synth.make_dout(w["B"], w["D"], w["T"] + 2, seed=4000)
+    g, ref = run_both(d, dout)
+    errs = check_grads(g, ref, TOL["bf16"], TOL["bf16"])
+    # fp32 arithmetic on exact bf16 inputs: far inside the bf16 bound
+    assert max(errs.values()) < 1e-3, errs
