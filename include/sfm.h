@@ -201,6 +201,43 @@ SFM_API sfm_status sfm_selective_scan_fold_bwd(const sfm_scan_args* args, const 
                                        sfm_stream_t stream);
 
 /*
+ * The scan backward without any allocation by the caller or the library.
+ *
+ * This entry point has no counterpart in the paper.  It is
+ * sfm_selective_scan_fold_bwd with its workspace taken from a buffer built into the
+ * library instead of one the caller passes in.  It is for callers that cannot call
+ * cudaMalloc, for example:
+ *   - a plug-in inside a host application that owns all device memory through its own
+ *     allocator and gives plug-ins no way to request more;
+ *   - a deployment that forbids allocation after start-up (a fixed memory budget
+ *     decided up front);
+ *   - a latency-critical loop where cudaMalloc's implicit device synchronisation is
+ *     not acceptable.
+ * The caller still passes every input and output tensor; only the workspace is built in.
+ *
+ * The built-in workspace is a device array of SFM_NOALLOC_SCRATCH_BYTES.  Every GPU that
+ * loads this library holds that much memory until the process exits.  Problems whose
+ * workspace (sfm_scan_bwd_workspace_size) exceeds it are rejected with
+ * SFM_ERR_UNSUPPORTED before anything is launched; use sfm_selective_scan_fold_bwd then.
+ *
+ * The first call on a device looks up the array's device address on that device
+ * (cudaGetSymbolAddress, with the device current); make that first call before any
+ * stream capture.  Later calls reuse the address.
+ *
+ * All calls on a device share the one array, and it keeps the last call's contents:
+ * the backward writes every part of the workspace before reading it, so nothing has to
+ * start at zero, but two calls that overlap on the GPU (different streams, or
+ * different host threads) race on it and give wrong results.  Serialise them.
+ *
+ * Arguments, requirements and results are exactly those of sfm_selective_scan_fold_bwd.
+ * No cudaMalloc, cudaFree or allocating library routine is called.
+ */
+#define SFM_NOALLOC_SCRATCH_BYTES (64u << 20) /* 64 MiB */
+SFM_API sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* args,
+                                                       const sfm_scan_grads* grads,
+                                                       sfm_stream_t stream);
+
+/*
  * Adaptive B1: the number of folded rows for a batch of B samples of T patch tokens,
  * D channels and state size N, from a look-up table built by a B200 sweep.  The
  * result always divides B.  Source: techloop.online, Adaptive B1; sungsoo.github.io

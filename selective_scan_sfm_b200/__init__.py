@@ -16,7 +16,7 @@ from ._abi import SFM_BF16, SFM_F32, SfmError
 
 __all__ = [
     "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d", "sfm_selective_scan_fold",
-    "sfm_selective_scan_fold_bwd", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
+    "sfm_selective_scan_fold_bwd", "sfm_selective_scan_fold_bwd_noalloc", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
     "SfmError", "library_path",
 ]
 
@@ -184,6 +184,26 @@ def sfm_selective_scan_fold_bwd(u, dt, Bm, Cm, A, dout, *, z=None, Dskip=None, d
     _abi.check(_abi.lib().sfm_selective_scan_fold_bwd(ctypes.byref(a), ctypes.byref(g),
                                                       ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
                                                       _stream(stream)), "sfm_selective_scan_fold_bwd")
+    return grads
+
+
+def sfm_selective_scan_fold_bwd_noalloc(u, dt, Bm, Cm, A, dout, grads, *, z=None, Dskip=None, dt_bias=None,
+                                        dt_softplus=True, stream=None):
+    """The scan backward with the workspace built into the library, for callers that
+    cannot allocate device memory (see include/sfm.h).  `grads` is a dict of
+    caller-allocated fp32 tensors (du, ddt, dA, dB, dC, and dz / dDskip / ddt_bias when
+    z / Dskip / dt_bias are given); it is filled in and returned."""
+    a, _ = _scan_args(u, dt, Bm, Cm, A, z, Dskip, dt_bias, None, None, None, None, 0, None, dt_softplus,
+                      False, False, None, 0, 0, 0, need_y=False)
+    _dev(dout, "dout", dt.dtype, (a.B, a.D, a.L))
+    g = _abi.ScanGrads()
+    g.size = ctypes.sizeof(_abi.ScanGrads)
+    g.dout = dout.data_ptr()
+    for k in ("du", "ddt", "dz", "dA", "dDskip", "ddt_bias", "dB", "dC"):
+        t = grads.get(k)
+        setattr(g, k, None if t is None else _dev(t, k, torch.float32).data_ptr())
+    _abi.check(_abi.lib().sfm_selective_scan_fold_bwd_noalloc(ctypes.byref(a), ctypes.byref(g), _stream(stream)),
+               "sfm_selective_scan_fold_bwd_noalloc")
     return grads
 
 

@@ -18,8 +18,11 @@ SFM_F32, SFM_BF16 = 0, 1
 ENTRY_POINTS = (
     "sfm_status_string", "sfm_abi_version", "sfm_last_cuda_error", "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d",
     "sfm_selective_scan_fold", "sfm_scan_bwd_workspace_size", "sfm_selective_scan_fold_bwd",
-    "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
+    "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error", "sfm_selective_scan_fold_bwd_noalloc",
 )
+
+#: Size of the workspace built into the library for sfm_selective_scan_fold_bwd_noalloc.
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -82,6 +85,7 @@ def lib():
         L.sfm_choose_b1.argtypes = [_i, _i, _i, _i, ctypes.POINTER(_i)]
         L.sfm_choose_variant.argtypes = [_i, _i, _i, _i, ctypes.POINTER(Variant)]
         L.sfm_get_device_error.argtypes = [_vp, _i, ctypes.POINTER(_i)]
+        L.sfm_selective_scan_fold_bwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanGrads), _vp]
         for name in ENTRY_POINTS:
             if name not in ("sfm_status_string", "sfm_abi_version", "sfm_last_cuda_error"):
                 getattr(L, name).restype = _i

@@ -357,6 +357,21 @@ sfm_status sfm_selective_scan_fold_bwd(const sfm_scan_args* a, const sfm_scan_gr
   return cuda_status(launch_bwd(p, a->in_dtype, a->out_dtype, stream));
 }
 
+sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* a, const sfm_scan_grads* g,
+                                               sfm_stream_t stream) {
+  sfm_status st = validate_bwd_args(a);
+  if (st != SFM_OK) return st;
+  if ((st = validate_grads(a, g)) != SFM_OK) return st;
+  if (bwd_workspace_bytes(a->B, a->D, a->L, a->N, kBwdDTile) > (size_t)SFM_NOALLOC_SCRATCH_BYTES)
+    return SFM_ERR_UNSUPPORTED;  // larger than the built-in workspace
+  if (fault_injected()) return SFM_ERR_CUDA;
+  void* ws = nullptr;
+  if ((st = cuda_status(noalloc_scratch(&ws))) != SFM_OK) return st;
+  BwdParams p = make_bwd_params(a, g);
+  bwd_carve(p, static_cast<char*>(ws));
+  return cuda_status(launch_bwd(p, a->in_dtype, a->out_dtype, stream));
+}
+
 sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code) {
   if (!code) return SFM_ERR_INVALID_ARG;
   unsigned v = 0;

@@ -16,6 +16,8 @@
 //     fixed order into per-tile partials.
 //   bwd_reduce_bc_kernel: dB, dC = sum of the tile partials, in tile order.
 //   bwd_reduce_param_kernel: dA, dDskip, ddt_bias = sum over samples, in sample order.
+#include <mutex>
+
 #include "sfm_device.cuh"
 #include "sfm_internal.h"
 
@@ -199,6 +201,31 @@ void bwd_carve(BwdParams& p, char* ws) {
   p.partA = take((size_t)p.B * p.D * p.N * 4);
   p.partD = take((size_t)p.B * p.D * 4);
   p.partBias = take((size_t)p.B * p.D * 4);
+}
+
+// Built-in workspace of sfm_selective_scan_fold_bwd_noalloc: a file-scope device array
+// that every GPU loading this library holds until the process exits.  Host code must not
+// pass its name to a kernel (on the host it is only a stand-in); noalloc_scratch() looks
+// up its device address once per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SFM_NOALLOC_SCRATCH_BYTES];
+
+cudaError_t noalloc_scratch(void** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {  // first call on this device (which is current): take the array's address
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
 }
 
 template <typename TI, typename TD>

@@ -75,6 +75,7 @@ cudaError_t read_device_error(cudaStream_t s, int clear, unsigned* value);
 cudaError_t launch_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dtype, cudaStream_t s);
 size_t bwd_workspace_bytes(int B, int D, int L, int N, int d_tile);
 void bwd_carve(BwdParams& p, char* ws);
+cudaError_t noalloc_scratch(void** out);  // device address of the built-in workspace
 
 cudaError_t launch_aux_init(const void* x, void* xa, int B, int D, int T, int esize, cudaStream_t s);
 cudaError_t launch_aux_swap(void* y, int B, int D, int L, int esize, cudaStream_t s);
