@@ -151,6 +151,8 @@ typedef struct {
   int lanes;            /* lanes per channel sequence (1 = one thread walks it)    */
   int d_tile;           /* channels per CTA (at most 128)                          */
   int chunk;            /* tokens staged per step of the walk                      */
+  int exp2_split;       /* 1 + state pairs per token whose exp2 runs on the FMA pipe
+                           instead of the transcendental unit (N = 16 only)        */
 } sfm_scan_args;
 
 /*
@@ -246,9 +248,10 @@ SFM_API sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* args
 SFM_API sfm_status sfm_choose_b1(int B, int T, int D, int N, int* B1_out);
 
 /* The full launch choice behind sfm_choose_b1: folded rows, lanes per channel
- * sequence, channels per CTA and tokens staged per step. */
+ * sequence, channels per CTA, tokens staged per step, and state pairs per token whose
+ * exp2 runs on the FMA pipe. */
 typedef struct {
-  int B1, lanes, d_tile, chunk;
+  int B1, lanes, d_tile, chunk, exp2_pairs;
 } sfm_variant;
 SFM_API sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* out);
 

@@ -16,7 +16,7 @@ using namespace sfm;
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 constexpr int kMaxDTile = 128;
 constexpr int kMaxChunk = 256;
 constexpr int kMaxB1 = 65535;  // grid.y
@@ -24,7 +24,7 @@ constexpr int kMaxNFused = 16;
 constexpr int kWholeSmemCap = 80 * 1024;  // whole-sample staging only while 2+ CTAs fit an SM
 
 struct LutEntry {
-  int T, B, D, N, B2, lanes, d_tile, chunk;
+  int T, B, D, N, B2, lanes, d_tile, chunk, exp2_pairs;
 };
 const LutEntry kLut[] = {
 #include "sfm_lut.inc"
@@ -96,7 +96,9 @@ sfm_variant choose(int B, int T, int D, int N) {
   int dt = best->d_tile;
   if (dt > round_up(D, 32)) dt = round_up(D, 32);
   v.d_tile = dt;
-  v.chunk = balanced_chunk(T + 2, best->chunk);
+  // the measured chunk for the row's own token count; re-balanced for other lengths
+  v.chunk = T == best->T ? best->chunk : balanced_chunk(T + 2, best->chunk);
+  v.exp2_pairs = N > 14 ? best->exp2_pairs : 0;
   return v;
 }
 
@@ -119,6 +121,7 @@ sfm_status validate_scan(const sfm_scan_args* a, bool bwd) {
   if (a->lanes < 0 || a->lanes > 1) return SFM_ERR_UNSUPPORTED;
   if (a->d_tile < 0 || a->d_tile > kMaxDTile) return SFM_ERR_UNSUPPORTED;
   if (a->chunk < 0 || a->chunk > kMaxChunk || (a->chunk % 8) != 0) return SFM_ERR_UNSUPPORTED;
+  if (a->exp2_split < 0 || a->exp2_split > 4) return SFM_ERR_UNSUPPORTED;
   const void* acts[] = {a->x, a->dt, a->z, a->Bm, a->Cm, a->y};
   for (const void* p : acts)
     if (p && !aligned16(p)) return SFM_ERR_MISALIGNED;
@@ -295,6 +298,7 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
   p.B2 = a->B / (a->B1 ? a->B1 : v.B1);
   p.d_tile = a->d_tile ? a->d_tile : v.d_tile;
   p.chunk = a->chunk ? a->chunk : v.chunk;
+  p.exp2_fma_pairs = a->exp2_split ? a->exp2_split - 1 : v.exp2_pairs;
   p.flags = (a->dt_softplus ? kSoftplus : 0) | (a->aux_init ? kAuxInit : 0) |
             (a->swap_out && a->L >= 2 ? kSwapOut : 0) | (a->conv_w ? kConv : 0) | (a->z ? kGate : 0);
   const int si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);

@@ -30,6 +30,62 @@ __device__ __forceinline__ float rcp(float x) {
   return y;
 }
 
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// ---- functions on the FMA pipe, to take load off the transcendental unit -------------
+// Coefficients: minimax polynomials fitted by the Remez exchange in
+// selective_scan_sfm_b200/poly_fit.py (fp32-rounded; the script reports their error).
+
+// 2^x for a pair of values.  Cody-Waite split x = j + f, j = round(x) (by adding and
+// subtracting 1.5*2^23), f in [-1/2, 1/2]; 2^f from a degree-5 polynomial (max relative
+// error 2.4e-7 in fp32, the accuracy of the hardware ex2.approx); 2^j is added into the
+// exponent field.  x is clamped to [-126, 126] so the result stays a normal number (a
+// NaN passes through the comparisons and stays NaN).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = x.x < -126.0f ? -126.0f : x.x;
+  x.y = x.y < -126.0f ? -126.0f : x.y;
+  x.x = x.x > 126.0f ? 126.0f : x.x;
+  x.y = x.y > 126.0f ? 126.0f : x.y;
+  const float2 M = make_float2(12582912.0f, 12582912.0f), mM = make_float2(-12582912.0f, -12582912.0f);
+  const float2 t = __fadd2_rn(x, M);
+  const float2 j = __fadd2_rn(t, mM);
+  const float2 f = __ffma2_rn(j, make_float2(-1.0f, -1.0f), x);
+  float2 p = __ffma2_rn(make_float2(1.327647245e-03f, 1.327647245e-03f), f,
+                        make_float2(9.675540961e-03f, 9.675540961e-03f));
+  p = __ffma2_rn(p, f, make_float2(5.550713092e-02f, 5.550713092e-02f));
+  p = __ffma2_rn(p, f, make_float2(2.402212024e-01f, 2.402212024e-01f));
+  p = __ffma2_rn(p, f, make_float2(6.931469440e-01f, 6.931469440e-01f));
+  p = __ffma2_rn(p, f, make_float2(1.000000119e+00f, 1.000000119e+00f));
+  p.x = __int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23));
+  p.y = __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23));
+  return p;
+}
+
+// softplus(v) = max(v, 0) + log(1 + w), w = e^-|v| in (0, 1], with log(1 + w) = w * q(w)
+// and q a degree-7 polynomial (max relative error 3.3e-7 in fp32): one transcendental.
+__device__ __forceinline__ float softplus_fast(float v) {
+  const float w = ex2(-fabsf(v) * kLog2e);
+  float q = fmaf(-8.539208211e-03f, w, 4.408963397e-02f);
+  q = fmaf(q, w, -1.076817140e-01f);
+  q = fmaf(q, w, 1.774524152e-01f);
+  q = fmaf(q, w, -2.449546307e-01f);
+  q = fmaf(q, w, 3.327547908e-01f);
+  q = fmaf(q, w, -4.999740422e-01f);
+  q = fmaf(q, w, 9.999998212e-01f);
+  return fmaxf(v, 0.0f) + w * q;
+}
+
+// SiLU(v) = v * (1 + tanh(v/2)) / 2 with the hardware tanh (relative error about 2^-11):
+// one transcendental instead of two.  Used only where the output is rounded to bf16.
+__device__ __forceinline__ float silu_fast(float v) {
+  const float h = 0.5f * v;
+  return fmaf(h, tanh_approx(h), h);
+}
+
 // SiLU(v) = v * sigmoid(v) = v / (1 + e^-v).  For e^-v = inf the reciprocal is 0.
 __device__ __forceinline__ float silu(float v) { return v * rcp(1.0f + ex2(-v * kLog2e)); }
 

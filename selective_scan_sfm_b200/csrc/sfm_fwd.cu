@@ -119,7 +119,9 @@ struct Chan {
 
 // State update and read-out of one token:
 //   h = Abar*h + Delta*B*u (Abar = 0 on a reset token), returns sum_n C_n h_n.
-template <int NH, bool RESET>
+// The exp2 of the first PE state pairs runs on the FMA pipe (exp2_fma2), the rest on the
+// transcendental unit, so that both pipes share the N exponentials.
+template <int NH, bool RESET, int PE>
 __device__ __forceinline__ float scan_token(Chan<NH>& c, const float* __restrict__ bc, float delta, float dbu) {
   const float2 d2 = make_float2(delta, delta), u2 = make_float2(dbu, dbu);
   float2 ya = make_float2(0.f, 0.f), yb = make_float2(0.f, 0.f);
@@ -144,8 +146,12 @@ __device__ __forceinline__ float scan_token(Chan<NH>& c, const float* __restrict
         c.h[k + j] = bu;
       } else {
         float2 a = __fmul2_rn(d2, c.A2[k + j]);
-        a.x = ex2(a.x);
-        a.y = ex2(a.y);
+        if (k + j < PE) {
+          a = exp2_fma2(a);
+        } else {
+          a.x = ex2(a.x);
+          a.y = ex2(a.y);
+        }
         c.h[k + j] = __ffma2_rn(a, c.h[k + j], bu);
       }
       if (j == 0)
@@ -166,7 +172,8 @@ struct Opts {
 
 // Output of one token from its conv taps (xw[0..3] = xa[t-pl .. t-pl+3]), raw dt and z.
 // STD: conv (K = 4) + softplus + gate, all compile-time; else the runtime options.
-template <typename TI, int NH, bool STD, bool RESET>
+// FAST: one-transcendental SiLU and softplus (used when the output is rounded to bf16).
+template <typename TI, int NH, bool STD, bool RESET, bool FAST, int PE>
 __device__ __forceinline__ float token_out(Chan<NH>& c, const Opts& o, const float* xw, TI dtv, TI zv,
                                            const float* __restrict__ bc) {
   float u;
@@ -175,15 +182,18 @@ __device__ __forceinline__ float token_out(Chan<NH>& c, const Opts& o, const flo
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       if (STD || q < o.K) acc = fmaf(c.w[q], xw[q], acc);
-    u = silu(acc);
+    u = FAST ? silu_fast(acc) : silu(acc);
   } else {
     u = xw[0];
   }
   const float v = to_f(dtv) + c.dtb;
-  const float delta = (STD || o.sp) ? softplus(v) : v;
-  float yv = scan_token<NH, RESET>(c, bc, delta, delta * u);
+  const float delta = (STD || o.sp) ? (FAST ? softplus_fast(v) : softplus(v)) : v;
+  float yv = scan_token<NH, RESET, PE>(c, bc, delta, delta * u);
   yv = fmaf(c.dsk, u, yv);
-  if (STD || o.gate) yv *= silu(to_f(zv));
+  if (STD || o.gate) {
+    const float zf = to_f(zv);
+    yv *= FAST ? silu_fast(zf) : silu(zf);
+  }
   return yv;
 }
 
@@ -201,21 +211,21 @@ __device__ __forceinline__ float xa_at(const Opts& o, const TI* xr, int xlo, int
 }
 
 // General path for token t (chunk-relative i): conv taps with explicit boundary handling.
-template <typename TI, typename TO, int NH, bool STD>
+template <typename TI, typename TO, int NH, bool STD, bool FAST, int PE>
 __device__ __forceinline__ float general_token(Chan<NH>& c, const Opts& o, const TI* xr, int xlo, int xhi, int t,
                                                TI dtv, TI zv, const float* bc) {
   float xw[4];
   const int K = (STD || o.conv) ? 4 : 1, pl = (STD || o.conv) ? o.pl : 0;
 #pragma unroll
   for (int q = 0; q < 4; ++q) xw[q] = q < K ? xa_at<TI>(o, xr, xlo, xhi, c.mean, t - pl + q) : 0.0f;
-  if (t == 0) return token_out<TI, NH, STD, true>(c, o, xw, dtv, zv, bc);
-  return token_out<TI, NH, STD, false>(c, o, xw, dtv, zv, bc);
+  if (t == 0) return token_out<TI, NH, STD, true, FAST, PE>(c, o, xw, dtv, zv, bc);
+  return token_out<TI, NH, STD, false, FAST, PE>(c, o, xw, dtv, zv, bc);
 }
 
 // G interior tokens starting at chunk-relative index i: loads first (x window, dt, z),
 // then the G token computations, then the stores, so the compiler can overlap tokens.
 // xb[i + q] is the conv tap q of token i (no boundary inside the group).
-template <typename TI, typename TO, int NH, bool STD, int G>
+template <typename TI, typename TO, int NH, bool STD, bool FAST, int PE, int G>
 __device__ __forceinline__ void fast_group(Chan<NH>& c, const Opts& o, const TI* __restrict__ xb,
                                            const TI* dtr, const TI* zr, TO* yr, int i,
                                            const float* __restrict__ bct) {
@@ -231,14 +241,15 @@ __device__ __forceinline__ void fast_group(Chan<NH>& c, const Opts& o, const TI*
   }
   float yv[G];
 #pragma unroll
-  for (int k = 0; k < G; ++k) yv[k] = token_out<TI, NH, STD, false>(c, o, xv + k, dv[k], zv[k], bct + (i + k) * NP2);
+  for (int k = 0; k < G; ++k)
+    yv[k] = token_out<TI, NH, STD, false, FAST, PE>(c, o, xv + k, dv[k], zv[k], bct + (i + k) * NP2);
 #pragma unroll
   for (int k = 0; k < G; ++k) yr[i + k] = from_f<TO>(yv[k]);
 }
 
 // Walks tokens [t0, t0 + cnt) of one sample.  xr: x row holding x indices [xlo, xhi);
 // dtr/zr/yr: rows indexed chunk-relative; bct: transposed B/C of the chunk.
-template <typename TI, typename TO, int NH, bool STD>
+template <typename TI, typename TO, int NH, bool STD, bool FAST, int PE>
 __device__ __forceinline__ void walk(Chan<NH>& c, const Opts& o, const TI* xr, int xlo, int xhi, const TI* dtr,
                                      const TI* zr, TO* yr, const float* bct, int t0, int cnt) {
   constexpr int NP2 = 4 * NH;
@@ -253,19 +264,20 @@ __device__ __forceinline__ void walk(Chan<NH>& c, const Opts& o, const TI* xr, i
   const int e2 = max(e1, min(tend, tb));
   for (int t = t0; t < e1; ++t) {
     const int i = t - t0;
-    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
+    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD, FAST, PE>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
   }
   if (e2 > e1) {
     // x index of tap 0 of token t is t - pl - off; xb[i + q] must be that + q
     const TI* xb = xr + (t0 - o.pl - o.off - xlo);
     int i = e1 - t0;
     const int iend = e2 - t0;
-    for (; i + kGroup <= iend; i += kGroup) fast_group<TI, TO, NH, STD, kGroup>(c, o, xb, dtr, zr, yr, i, bct);
-    for (; i < iend; ++i) fast_group<TI, TO, NH, STD, 1>(c, o, xb, dtr, zr, yr, i, bct);
+    for (; i + kGroup <= iend; i += kGroup)
+      fast_group<TI, TO, NH, STD, FAST, PE, kGroup>(c, o, xb, dtr, zr, yr, i, bct);
+    for (; i < iend; ++i) fast_group<TI, TO, NH, STD, FAST, PE, 1>(c, o, xb, dtr, zr, yr, i, bct);
   }
   for (int t = e2; t < tend; ++t) {
     const int i = t - t0;
-    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
+    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD, FAST, PE>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
   }
 }
 
@@ -340,9 +352,10 @@ __device__ __forceinline__ Opts make_opts(const FwdParams& p) {
 // ------------------------------------------------------------------ whole-sample mode
 
 // Shared memory: [barrier 16 B][x slab][dt slab][z slab][B][C][bct][y slab if not in place]
-template <typename TI, typename TO, int NH, bool STD>
+template <typename TI, typename TO, int NH, bool STD, int PE>
 __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
   constexpr bool kInPlace = std::is_same<TI, TO>::value;
+  constexpr bool kFast = std::is_same<TO, __nv_bfloat16>::value;
   constexpr int si = sizeof(TI), so = sizeof(TO), NP = 2 * NH;
   extern __shared__ __align__(16) char smem[];
 
@@ -421,7 +434,7 @@ __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
       TO* yr = kInPlace ? reinterpret_cast<TO*>(dts) + tid * L : reinterpret_cast<TO*>(ys) + tid * L;
 #pragma unroll
       for (int k = 0; k < NH; ++k) c.h[k] = make_float2(0.f, 0.f);
-      walk<TI, TO, NH, STD>(c, o, xr, 0, Tx, dtr, zr, yr, bct, 0, L);
+      walk<TI, TO, NH, STD, kFast, PE>(c, o, xr, 0, Tx, dtr, zr, yr, bct, 0, L);
       if (swap) {
         const TO h0 = yr[0];
         yr[0] = yr[L - 1];
@@ -448,9 +461,10 @@ __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
 
 // ------------------------------------------------------------------ chunked mode
 
-template <typename TI, typename TO, int NH, bool STD>
+template <typename TI, typename TO, int NH, bool STD, int PE>
 __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
   constexpr bool kInPlace = std::is_same<TI, TO>::value;
+  constexpr bool kFast = std::is_same<TO, __nv_bfloat16>::value;
   constexpr int si = sizeof(TI), so = sizeof(TO), NP = 2 * NH;
   extern __shared__ __align__(16) char smem[];
 
@@ -527,7 +541,7 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
         const TI* dtr = reinterpret_cast<const TI*>(dts + tid * p.io_row + hd);
         const TI* zr = o.gate ? reinterpret_cast<const TI*>(zs + tid * p.io_row + hd) : dtr;
         TO* yr = kInPlace ? reinterpret_cast<TO*>(dts + tid * p.io_row + hd) : reinterpret_cast<TO*>(ys + tid * p.y_row);
-        walk<TI, TO, NH, STD>(c, o, xr, xlo, xhi, dtr, zr, yr, bct, t0, cnt);
+        walk<TI, TO, NH, STD, kFast, PE>(c, o, xr, xlo, xhi, dtr, zr, yr, bct, t0, cnt);
         if (swap) {
           if (t0 == 0) head_val = yr[0];  // goes to position L-1
           if (t0 + cnt == L) {
@@ -601,26 +615,37 @@ static cudaError_t set_smem(Kern k, int bytes, int& have) {
   return e;
 }
 
-template <typename TI, typename TO, int NH, bool STD>
+template <typename TI, typename TO, int NH, bool STD, int PE>
 static cudaError_t launch_t(const FwdParams& p, cudaStream_t s) {
   static int whole_set = 48 * 1024, chunk_set = 48 * 1024;
   const int threads = (p.d_tile + 31) & ~31;
   dim3 grid((p.D + p.d_tile - 1) / p.d_tile, p.B / p.B2);
   cudaError_t e;
   if (p.mode == kModeWhole) {
-    if ((e = set_smem(fwd_whole_kernel<TI, TO, NH, STD>, p.smem_bytes, whole_set)) != cudaSuccess) return e;
-    fwd_whole_kernel<TI, TO, NH, STD><<<grid, threads, p.smem_bytes, s>>>(p);
+    if ((e = set_smem(fwd_whole_kernel<TI, TO, NH, STD, PE>, p.smem_bytes, whole_set)) != cudaSuccess) return e;
+    fwd_whole_kernel<TI, TO, NH, STD, PE><<<grid, threads, p.smem_bytes, s>>>(p);
   } else {
-    if ((e = set_smem(fwd_chunk_kernel<TI, TO, NH, STD>, p.smem_bytes, chunk_set)) != cudaSuccess) return e;
-    fwd_chunk_kernel<TI, TO, NH, STD><<<grid, threads, p.smem_bytes, s>>>(p);
+    if ((e = set_smem(fwd_chunk_kernel<TI, TO, NH, STD, PE>, p.smem_bytes, chunk_set)) != cudaSuccess) return e;
+    fwd_chunk_kernel<TI, TO, NH, STD, PE><<<grid, threads, p.smem_bytes, s>>>(p);
   }
   return cudaGetLastError();
 }
 
+// The standard mixer (conv K=4 + softplus + gate) gets the specialised path and, at
+// N = 16, a choice of how many state pairs take exp2 on the FMA pipe.
 template <typename TI, typename TO, int NH>
 static cudaError_t launch_std(const FwdParams& p, cudaStream_t s) {
   const bool std_path = (p.flags & kConv) && (p.flags & kGate) && (p.flags & kSoftplus) && p.K == 4;
-  return std_path ? launch_t<TI, TO, NH, true>(p, s) : launch_t<TI, TO, NH, false>(p, s);
+  if (!std_path) return launch_t<TI, TO, NH, false, 0>(p, s);
+  if constexpr (NH == 8) {
+    switch (p.exp2_fma_pairs) {
+      case 1: return launch_t<TI, TO, NH, true, 1>(p, s);
+      case 2: return launch_t<TI, TO, NH, true, 2>(p, s);
+      case 3: return launch_t<TI, TO, NH, true, 3>(p, s);
+      default: break;
+    }
+  }
+  return launch_t<TI, TO, NH, true, 0>(p, s);
 }
 
 template <typename TI, typename TO>

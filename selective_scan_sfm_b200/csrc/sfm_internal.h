@@ -36,6 +36,7 @@ struct FwdParams {
   int chunk;           // tokens staged per step of the walk
   int flags;
   int mode;            // kModeWhole or kModeChunk
+  int exp2_fma_pairs;  // state pairs per token whose exp2 runs on the FMA pipe (N = 16 path)
   // shared-memory carve-up (bytes), computed on the host
   int x_row, io_row, y_row, smem_bytes;
 };
