@@ -74,18 +74,37 @@ def algorithmic_bytes(B, D, T, L, N, K, in_size, out_size):
     return acts + params + B * D * L * out_size
 
 
+POLY_EXP2_FMA_OPS = 8      # FMA-pipe lane-ops of one polynomial exp2 (Cody-Waite + degree 5)
+
+
 def alu_ops_per_element(N, K):
-    """(transcendentals, fp32 ops) per element of the fused forward.
-    Transcendentals: N decays exp(Delta*A_n); softplus (exp, log); SiLU of the conv
-    output and of z (exp, reciprocal each).  FP32: 4 per state (Delta*A, Delta*B*u,
-    state update, read-out) plus conv K, softplus 8, two SiLU 2x2, skip, gate, Delta*u."""
-    return N + 6, 4 * N + K + 8 + 4 + 3
+    """(transcendental functions, fp32 ops) per element of the fused forward.
+    Transcendentals: N decays exp(Delta*A_n); softplus (an exp and a log); the two SiLUs
+    (one sigmoid each).  FP32: 4 per state (Delta*A, B*Delta*u, state update, read-out),
+    the conv (K taps + bias), Delta*u, the D skip, the gate, and about 6 around the
+    transcendentals."""
+    return N + 4, 4 * N + K + 12
+
+
+def alu_clk_per_element(N, K):
+    """Least SM clocks per element on the two pipes that can do the work: each
+    transcendental goes either to the MUFU (16 lanes/clk/SM) or, as a polynomial of
+    POLY_EXP2_FMA_OPS lane-ops, to the FMA pipe (128 lanes/clk/SM) that also carries the
+    fp32 work; the best split balances the two pipes."""
+    E, F = alu_ops_per_element(N, K)
+    c = POLY_EXP2_FMA_OPS
+    m = (F + c * E) / (FP32_PER_CLK_SM / MUFU_PER_CLK_SM + c)  # transcendentals left on the MUFU
+    m = min(max(m, 0.0), E)
+    return max(m / MUFU_PER_CLK_SM, (F + c * (E - m)) / FP32_PER_CLK_SM)
 
 
 def alu_peak_elems(N, K, sm_mhz, sms=SMS):
-    tr, fp = alu_ops_per_element(N, K)
-    clk = max(tr / MUFU_PER_CLK_SM, fp / FP32_PER_CLK_SM)
-    return sms * sm_mhz * 1e6 / clk
+    return sms * sm_mhz * 1e6 / alu_clk_per_element(N, K)
+
+
+def mufu_only_peak_elems(N, K, sm_mhz, sms=SMS):
+    E, F = alu_ops_per_element(N, K)
+    return sms * sm_mhz * 1e6 / max(E / MUFU_PER_CLK_SM, F / FP32_PER_CLK_SM)
 
 
 def kernel_source_hash():
@@ -445,8 +464,11 @@ def main(argv=None):
         "roofline": {"bound": "alu", "achieved": elem_rate / 1e9, "peak": alu_peak / 1e9, "unit": "Gelem/s",
                      "frac": elem_rate / alu_peak, "traffic": recorded_traffic(args.workload),
                      "peak_basis": "%d MUFU + %d FP32 lanes/clk/SM x %d SMs x %.0f MHz; %d transcendentals and "
-                                   "%d fp32 ops per element" % ((MUFU_PER_CLK_SM, FP32_PER_CLK_SM, SMS, sm_max)
-                                                                + alu_ops_per_element(w["N"], w["K"]))},
+                                   "%d fp32 ops per element, a transcendental costing 1 MUFU lane or %d FMA-pipe "
+                                   "lane-ops, best split" % ((MUFU_PER_CLK_SM, FP32_PER_CLK_SM, SMS, sm_max)
+                                                             + alu_ops_per_element(w["N"], w["K"])
+                                                             + (POLY_EXP2_FMA_OPS,)),
+                     "peak_mufu_only": mufu_only_peak_elems(w["N"], w["K"], sm_max) / 1e9},
         "hbm": {"achieved": hbm_achieved, "peak": hbm_peak, "unit": "GB/s", "frac": hbm_achieved / hbm_peak,
                 "peak_source": peak_src, "algorithmic_bytes_per_launch": res["bytes"]},
         "kernel_ms": launch_ms,

@@ -92,9 +92,14 @@ sfm_variant choose(int B, int T, int D, int N) {
     B2 = next;
   }
   v.B1 = B / B2;
-  v.lanes = 1;
+  v.lanes = best->lanes > 1 ? best->lanes : 1;
   int dt = best->d_tile;
-  if (dt > round_up(D, 32)) dt = round_up(D, 32);
+  if (v.lanes > 1) {  // lanes mode: d_tile * lanes threads, a multiple of 32, at most 256
+    if (dt * v.lanes > 256) dt = 256 / v.lanes;
+    if (dt * v.lanes < 32) dt = 32 / v.lanes;
+  } else if (dt > round_up(D, 32)) {
+    dt = round_up(D, 32);
+  }
   v.d_tile = dt;
   // the measured chunk for the row's own token count; re-balanced for other lengths
   v.chunk = T == best->T ? best->chunk : balanced_chunk(T + 2, best->chunk);
@@ -118,7 +123,9 @@ sfm_status validate_scan(const sfm_scan_args* a, bool bwd) {
   if (a->reset_period != 0 && a->reset_period != a->L) return SFM_ERR_UNSUPPORTED;
   if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SFM_ERR_INVALID_ARG;
   if (a->in_dtype == SFM_F32 && a->out_dtype == SFM_BF16) return SFM_ERR_UNSUPPORTED;
-  if (a->lanes < 0 || a->lanes > 1) return SFM_ERR_UNSUPPORTED;
+  if (a->lanes < 0 || a->lanes > 32 || (a->lanes & (a->lanes - 1)) != 0) return SFM_ERR_UNSUPPORTED;
+  if (a->lanes > 1 && a->d_tile && (a->d_tile * a->lanes > 256 || (a->d_tile * a->lanes) % 32 != 0))
+    return SFM_ERR_UNSUPPORTED;
   if (a->d_tile < 0 || a->d_tile > kMaxDTile) return SFM_ERR_UNSUPPORTED;
   if (a->chunk < 0 || a->chunk > kMaxChunk || (a->chunk % 8) != 0) return SFM_ERR_UNSUPPORTED;
   if (a->exp2_split < 0 || a->exp2_split > 4) return SFM_ERR_UNSUPPORTED;
@@ -315,7 +322,22 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
   const bool aligned = slab_ok((long long)p.Tx * si) && slab_ok((long long)a->L * si) &&
                        slab_ok((long long)a->L * so) && ((long long)a->N * a->L * si) % 16 == 0;
   p.mode = kModeChunk;
-  if (p.chunk >= a->L && aligned) {
+  // an explicit channel tile or chunk without explicit lanes asks for one thread per channel
+  p.lanes = a->lanes ? a->lanes : ((a->d_tile || a->chunk) ? 1 : v.lanes);
+  if (p.lanes > 1) {
+    p.mode = kModeLanes;
+    if (!a->d_tile) {
+      if (p.d_tile * p.lanes > 256) p.d_tile = 256 / p.lanes;
+      if (p.d_tile * p.lanes < 32) p.d_tile = 32 / p.lanes;
+    }
+    if (p.d_tile * p.lanes > 256 || (p.d_tile * p.lanes) % 32 != 0) return SFM_ERR_UNSUPPORTED;
+    p.chunk = p.lanes * kLaneTokens;
+    p.x_row = fwd_x_row(p.chunk, 4, si);
+    p.io_row = fwd_io_row(p.chunk, si);
+    p.y_row = fwd_y_row(p.chunk, so);
+    p.smem_bytes = fwd_lanes_smem(p, si, so, NP);
+    if (p.smem_bytes > fwd_max_smem()) return SFM_ERR_UNSUPPORTED;
+  } else if (p.chunk >= a->L && aligned) {
     p.mode = kModeWhole;
     p.smem_bytes = fwd_whole_smem(p, si, so, NP);
     if (p.smem_bytes > kWholeSmemCap) p.mode = kModeChunk;

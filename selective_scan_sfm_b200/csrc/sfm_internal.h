@@ -35,7 +35,8 @@ struct FwdParams {
   int d_tile;          // channels per CTA (= threads per CTA for one lane per channel)
   int chunk;           // tokens staged per step of the walk
   int flags;
-  int mode;            // kModeWhole or kModeChunk
+  int mode;            // kModeWhole, kModeChunk or kModeLanes
+  int lanes;           // lanes per channel in kModeLanes (chunk = lanes * 8)
   int exp2_fma_pairs;  // state pairs per token whose exp2 runs on the FMA pipe (N = 16 path)
   // shared-memory carve-up (bytes), computed on the host
   int x_row, io_row, y_row, smem_bytes;
@@ -44,6 +45,8 @@ struct FwdParams {
 // Staging modes of the forward kernel: whole-sample slabs by bulk copy, or token chunks.
 constexpr int kModeChunk = 0;
 constexpr int kModeWhole = 1;
+constexpr int kModeLanes = 2;  // P lanes per channel split the tokens (warp-shuffle scan)
+constexpr int kLaneTokens = 8; // tokens per lane per chunk in kModeLanes
 
 struct BwdParams {
   const void* u;
@@ -67,6 +70,7 @@ struct BwdParams {
 cudaError_t launch_fwd(const FwdParams& p, sfm_dtype in_dtype, sfm_dtype out_dtype, int NP, cudaStream_t s);
 int fwd_whole_smem(const FwdParams& p, int in_size, int out_size, int NP);
 int fwd_chunk_smem(const FwdParams& p, int in_size, int out_size, int NP);
+int fwd_lanes_smem(const FwdParams& p, int in_size, int out_size, int NP);
 int fwd_max_smem();
 int fwd_x_row(int chunk, int K, int esize);
 int fwd_io_row(int chunk, int esize);

@@ -40,20 +40,26 @@ def divisors_upto(B, cap):
 
 
 def candidates(B, T, D):
+    """(B2, d_tile, chunk, lanes): one thread per channel (lanes = 1) with whole-sample or
+    chunked staging, and, for longer samples, P lanes per channel (chunk = 8 P)."""
     L = T + 2
     out = []
     tiles = [t for t in (32, 64, 128) if t <= max(32, ((D + 31) // 32) * 32)]
     chunks = sorted(set([c for c in (32, 56, 64, 128) if c < L] + [((L + 7) // 8) * 8 if L <= 256 else 0]) - {0})
     for B2, dt, ch in itertools.product(divisors_upto(B, 32), tiles, chunks):
-        out.append((B2, dt, ch))
+        out.append((B2, dt, ch, 1))
+    if L >= 100:
+        for B2, P, threads in itertools.product(divisors_upto(B, 4), (2, 4, 8, 16, 32), (64, 128, 256)):
+            if threads // P >= 1 and 8 * P <= 4 * L:
+                out.append((B2, threads // P, 8 * P, P))
     return out
 
 
-def time_variant(sets, lib, stream, B2, d_tile, chunk, reps, exp2_split=0):
+def time_variant(sets, lib, stream, B2, d_tile, chunk, reps, exp2_split=0, lanes=1):
     args = []
     for s in sets:
         a = s["args"]
-        a.B1, a.d_tile, a.chunk, a.exp2_split = s["B"] // B2, d_tile, chunk, exp2_split
+        a.B1, a.d_tile, a.chunk, a.exp2_split, a.lanes = s["B"] // B2, d_tile, chunk, exp2_split, lanes
         args.append(ctypes.byref(a))
     sp = ctypes.c_void_p(stream.cuda_stream)
     for i in range(3):
@@ -92,17 +98,17 @@ def sweep(grid, reps=15, log=print):
             sets.append(dict(args=a, keep=(dc, y), B=B))
         rows = []
         split0 = 3 if N == 16 else 1  # stage 1 at two FMA-pipe exp2 pairs (N = 16)
-        for (B2, dtile, ch) in candidates(B, T, D):
-            ms = time_variant(sets, lib, stream, B2, dtile, ch, reps, split0)
+        for (B2, dtile, ch, P) in candidates(B, T, D):
+            ms = time_variant(sets, lib, stream, B2, dtile, ch, reps, split0, P)
             if ms is None:
                 continue
-            rows.append(dict(B2=B2, d_tile=dtile, chunk=ch, exp2_pairs=split0 - 1, ms=ms,
+            rows.append(dict(B2=B2, d_tile=dtile, chunk=ch, lanes=P, exp2_pairs=split0 - 1, ms=ms,
                              gelem_s=B * D * (T + 2) / ms / 1e6))
         rows.sort(key=lambda r: r["ms"])
-        if N == 16:  # stage 2: the exp2 split for the best launch shape
+        if N == 16 and rows[0]["lanes"] == 1:  # stage 2: the exp2 split for the best launch shape
             b0 = rows[0]
             for split in (1, 2, 4):
-                ms = time_variant(sets, lib, stream, b0["B2"], b0["d_tile"], b0["chunk"], reps, split)
+                ms = time_variant(sets, lib, stream, b0["B2"], b0["d_tile"], b0["chunk"], reps, split, 1)
                 if ms is not None:
                     rows.append(dict(b0, exp2_pairs=split - 1, ms=ms, gelem_s=B * D * (T + 2) / ms / 1e6))
             rows.sort(key=lambda r: r["ms"])
@@ -110,25 +116,25 @@ def sweep(grid, reps=15, log=print):
         unfolded = min((r for r in rows if r["B2"] == 1), key=lambda r: r["ms"])
         res = dict(T=T, B=B, D=D, N=N, dtype=dtype, best=best, best_unfolded=unfolded, all=rows)
         results.append(res)
-        log("T=%4d B=%4d D=%5d N=%2d best B2=%2d d_tile=%3d chunk=%3d exp2_pairs=%d %.4f ms (%.1f Gelem/s); "
-            "best unfolded %.4f ms -> folding speedup %.3f" % (T, B, D, N, best["B2"], best["d_tile"], best["chunk"],
-                                                                best["exp2_pairs"], best["ms"], best["gelem_s"],
-                                                                unfolded["ms"], unfolded["ms"] / best["ms"]))
+        log("T=%4d B=%4d D=%5d N=%2d best B2=%2d lanes=%2d d_tile=%3d chunk=%3d exp2_pairs=%d %.4f ms "
+            "(%.1f Gelem/s); best unfolded %.4f ms -> folding speedup %.3f" % (
+                T, B, D, N, best["B2"], best["lanes"], best["d_tile"], best["chunk"], best["exp2_pairs"], best["ms"],
+                best["gelem_s"], unfolded["ms"], unfolded["ms"] / best["ms"]))
         del sets
         torch.cuda.empty_cache()
     return results
 
 
-def write_lut(results, path=LUT):
-    gpu = torch.cuda.get_device_name()
+def write_lut(results, path=LUT, gpu=None):
+    gpu = gpu or results[0].get("gpu") or torch.cuda.get_device_name()
     lines = ["// sfm_lut.inc -- adaptive-B1 look-up table: launch choices measured on B200.",
              "// Written by selective_scan_sfm_b200/lut_sweep.py from a sweep over B, T, D and N on %s;" % gpu,
              "// each row is the fastest measured variant for that shape.",
              "// Columns: T, B, D, N, B2, lanes, d_tile, chunk, exp2_pairs."]
     for r in results:
         b = r["best"]
-        lines.append("{%d, %d, %d, %d, %d, 1, %d, %d, %d}," % (r["T"], r["B"], r["D"], r["N"], b["B2"], b["d_tile"],
-                                                              b["chunk"], b["exp2_pairs"]))
+        lines.append("{%d, %d, %d, %d, %d, %d, %d, %d, %d}," % (r["T"], r["B"], r["D"], r["N"], b["B2"], b["lanes"],
+                                                               b["d_tile"], b["chunk"], b["exp2_pairs"]))
     open(path, "w").write("\n".join(lines) + "\n")
 
 
@@ -138,8 +144,14 @@ def main():
     ap.add_argument("--write", action="store_true")
     ap.add_argument("--json", default=None)
     ap.add_argument("--reps", type=int, default=15)
+    ap.add_argument("--from-json", default=None, help="rewrite the table from a saved sweep (no GPU needed)")
     a = ap.parse_args()
+    if a.from_json:
+        write_lut(json.load(open(a.from_json)))
+        return
     res = sweep(GRID_QUICK if a.quick else GRID_FULL, reps=a.reps)
+    for r in res:
+        r["gpu"] = torch.cuda.get_device_name()
     if a.json:
         json.dump(res, open(a.json, "w"), indent=1)
     if a.write:

@@ -221,3 +221,51 @@ def test_chain_of_four_layers():
         check(y[samples], ref, "bf16", "chain layer %d" % i)
         x = y
         xo = torch.from_numpy(bf16_round(ref)).to(torch.bfloat16)
+
+
+# ------------------------------------------------------------------ lanes mode: P lanes split a channel's tokens
+
+LANES_GRID = [
+    # B, D, T, N, dtype, lanes, d_tile
+    (2, 40, 300, 16, "bf16", 8, 16),
+    (3, 20, 130, 8, "f32", 4, 8),
+    (2, 33, 100, 5, "f32", 16, 2),
+    (1, 8, 500, 16, "bf16", 32, 4),
+    (4, 64, 75, 16, "bf16", 2, 64),
+    (2, 10, 17, 1, "f32", 8, 4),
+    (2, 12, 61, 3, "f32", 32, 8),
+]
+
+
+@pytest.mark.parametrize("B,D,T,N,dtype,lanes,d_tile", LANES_GRID)
+def test_lanes_against_oracle(B, D, T, N, dtype, lanes, d_tile):
+    d = synth.make_inputs(B=B, D=D, T=T, N=N, dtype=dtype, seed=7000 + T + lanes, random_A=True)
+    dc = to_cuda(d)
+    for swap in (False, True):
+        fs = torch.full((B, D, N), float("nan"), device="cuda")
+        y = fused(dc, swap_out=swap, lanes=lanes, d_tile=d_tile, B1=B, final_state=fs)
+        ref, ref_state = oracle_layer(d, swap_out=swap, want_state=True)
+        check(y, ref, dtype, "lanes=%d swap=%s" % (lanes, swap))
+        assert rel_err(fs.double().cpu().numpy(), ref_state) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("conv,gate,aux", [(False, False, False), (True, False, True), (False, True, True)])
+def test_lanes_optional_parts(conv, gate, aux):
+    d = synth.make_inputs(B=2, D=24, T=90, N=8, dtype="f32", seed=7100, aux=aux)
+    dc = to_cuda(d)
+    y = sfm_selective_scan_fold(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], z=dc["z"] if gate else None,
+                                Dskip=dc["Dskip"], dt_bias=dc["dt_bias"], conv_w=dc["conv_w"] if conv else None,
+                                conv_b=dc["conv_b"] if conv else None, aux_init=aux, lanes=8, d_tile=8)
+    check(y, oracle_layer(d, aux_init=aux, conv=conv, gate=gate), "f32")
+
+
+def test_lanes_sample_isolation():
+    d = synth.make_inputs(B=4, D=16, T=200, N=16, dtype="bf16", seed=7200)
+    dc = to_cuda(d)
+    y0 = fused(dc, lanes=8, d_tile=16, B1=1)
+    for field in ("x", "dt", "Bm"):
+        p = dict(dc)
+        p[field] = dc[field].clone()
+        p[field][1] = float("nan")
+        y1 = fused(p, lanes=8, d_tile=16, B1=1)
+        assert torch.equal(y1[[0, 2, 3]], y0[[0, 2, 3]]), field
