@@ -153,6 +153,8 @@ typedef struct {
   int chunk;            /* tokens staged per step of the walk                      */
   int exp2_split;       /* 1 + state pairs per token whose exp2 runs on the FMA pipe
                            instead of the transcendental unit (N = 16 only)        */
+  int chans_per_thread; /* channels one thread walks side by side (1 or 2; 2 needs the
+                           standard mixer at 8 < N <= 16, even D and d_tile)      */
 } sfm_scan_args;
 
 /*
@@ -248,10 +250,10 @@ SFM_API sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* args
 SFM_API sfm_status sfm_choose_b1(int B, int T, int D, int N, int* B1_out);
 
 /* The full launch choice behind sfm_choose_b1: folded rows, lanes per channel
- * sequence, channels per CTA, tokens staged per step, and state pairs per token whose
- * exp2 runs on the FMA pipe. */
+ * sequence, channels per CTA, tokens staged per step, state pairs per token whose
+ * exp2 runs on the FMA pipe, and channels per thread. */
 typedef struct {
-  int B1, lanes, d_tile, chunk, exp2_pairs;
+  int B1, lanes, d_tile, chunk, exp2_pairs, chans_per_thread;
 } sfm_variant;
 SFM_API sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* out);
 

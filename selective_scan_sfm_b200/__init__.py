@@ -96,7 +96,7 @@ def sfm_fold_conv1d(x, w, bias=None, u=None, pad_left=None, B2=1, silu=False, st
 
 
 def _scan_args(x, dt, Bm, Cm, A, z, Dskip, dt_bias, conv_w, conv_b, y, final_state, B1, pad_left, dt_softplus,
-               aux_init, swap_out, out_dtype, lanes, d_tile, chunk, need_y=True, exp2_split=0):
+               aux_init, swap_out, out_dtype, lanes, d_tile, chunk, need_y=True, exp2_split=0, chans_per_thread=0):
     _dev(dt, "dt")
     B, D, L = dt.shape
     io = dt.dtype
@@ -136,17 +136,20 @@ def _scan_args(x, dt, Bm, Cm, A, z, Dskip, dt_bias, conv_w, conv_b, y, final_sta
     a.dt_softplus, a.aux_init, a.swap_out = int(bool(dt_softplus)), int(bool(aux_init)), int(bool(swap_out))
     a.in_dtype, a.out_dtype = _code(io), _code(od)
     a.lanes, a.d_tile, a.chunk, a.exp2_split = int(lanes), int(d_tile), int(chunk), int(exp2_split)
+    a.chans_per_thread = int(chans_per_thread)
     return a, y
 
 
 def sfm_selective_scan_fold(x, dt, Bm, Cm, A, *, z=None, Dskip=None, dt_bias=None, conv_w=None, conv_b=None,
                             y=None, final_state=None, B1=0, pad_left=None, dt_softplus=True, aux_init=False,
-                            swap_out=False, out_dtype=None, lanes=0, d_tile=0, chunk=0, exp2_split=0, stream=None):
+                            swap_out=False, out_dtype=None, lanes=0, d_tile=0, chunk=0, exp2_split=0,
+                            chans_per_thread=0, stream=None):
     """Fused forward: [aux init] -> conv+SiLU -> folded scan with reset -> D skip ->
-    SiLU(z) gate -> [aux swap].  Returns y [B,D,L].  B1, d_tile, chunk, exp2_split:
-    launch-shape overrides (0 = the look-up table's choice)."""
+    SiLU(z) gate -> [aux swap].  Returns y [B,D,L].  B1, lanes, d_tile, chunk, exp2_split,
+    chans_per_thread: launch-shape overrides (0 = the look-up table's choice)."""
     a, y = _scan_args(x, dt, Bm, Cm, A, z, Dskip, dt_bias, conv_w, conv_b, y, final_state, B1, pad_left,
-                      dt_softplus, aux_init, swap_out, out_dtype, lanes, d_tile, chunk, exp2_split=exp2_split)
+                      dt_softplus, aux_init, swap_out, out_dtype, lanes, d_tile, chunk, exp2_split=exp2_split,
+                      chans_per_thread=chans_per_thread)
     _abi.check(_abi.lib().sfm_selective_scan_fold(ctypes.byref(a), _stream(stream)), "sfm_selective_scan_fold")
     return y
 
@@ -211,7 +214,8 @@ def sfm_selective_scan_fold_bwd_noalloc(u, dt, Bm, Cm, A, dout, grads, *, z=None
 def sfm_choose_variant(B: int, T: int, D: int, N: int) -> dict:
     v = _abi.Variant()
     _abi.check(_abi.lib().sfm_choose_variant(int(B), int(T), int(D), int(N), ctypes.byref(v)), "sfm_choose_variant")
-    return dict(B1=v.B1, lanes=v.lanes, d_tile=v.d_tile, chunk=v.chunk, exp2_pairs=v.exp2_pairs)
+    return dict(B1=v.B1, lanes=v.lanes, d_tile=v.d_tile, chunk=v.chunk, exp2_pairs=v.exp2_pairs,
+                chans_per_thread=v.chans_per_thread)
 
 
 def sfm_choose_b1(B: int, T: int, D: int, N: int) -> int:

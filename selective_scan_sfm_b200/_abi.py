@@ -40,7 +40,7 @@ class ScanArgs(ctypes.Structure):
         ("B1", _i), ("reset_period", _i),
         ("dt_softplus", _i), ("aux_init", _i), ("swap_out", _i),
         ("in_dtype", _i), ("out_dtype", _i),
-        ("lanes", _i), ("d_tile", _i), ("chunk", _i), ("exp2_split", _i),
+        ("lanes", _i), ("d_tile", _i), ("chunk", _i), ("exp2_split", _i), ("chans_per_thread", _i),
     ]
 
 
@@ -55,7 +55,8 @@ class ScanGrads(ctypes.Structure):
 
 class Variant(ctypes.Structure):
     """Mirror of sfm_variant."""
-    _fields_ = [("B1", _i), ("lanes", _i), ("d_tile", _i), ("chunk", _i), ("exp2_pairs", _i)]
+    _fields_ = [("B1", _i), ("lanes", _i), ("d_tile", _i), ("chunk", _i), ("exp2_pairs", _i),
+                ("chans_per_thread", _i)]
 
 
 _lib = None

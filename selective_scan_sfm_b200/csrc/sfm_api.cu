@@ -16,7 +16,7 @@ using namespace sfm;
 
 namespace {
 
-constexpr int kAbiVersion = 2;
+constexpr int kAbiVersion = 3;
 constexpr int kMaxDTile = 128;
 constexpr int kMaxChunk = 256;
 constexpr int kMaxB1 = 65535;  // grid.y
@@ -24,7 +24,7 @@ constexpr int kMaxNFused = 16;
 constexpr int kWholeSmemCap = 80 * 1024;  // whole-sample staging only while 2+ CTAs fit an SM
 
 struct LutEntry {
-  int T, B, D, N, B2, lanes, d_tile, chunk, exp2_pairs;
+  int T, B, D, N, B2, lanes, d_tile, chunk, exp2_pairs, cpt;
 };
 const LutEntry kLut[] = {
 #include "sfm_lut.inc"
@@ -104,6 +104,7 @@ sfm_variant choose(int B, int T, int D, int N) {
   // the measured chunk for the row's own token count; re-balanced for other lengths
   v.chunk = T == best->T ? best->chunk : balanced_chunk(T + 2, best->chunk);
   v.exp2_pairs = N > 14 ? best->exp2_pairs : 0;
+  v.chans_per_thread = (best->cpt == 2 && N > 8 && N <= 16 && D % 2 == 0 && v.lanes == 1) ? 2 : 1;
   return v;
 }
 
@@ -129,6 +130,7 @@ sfm_status validate_scan(const sfm_scan_args* a, bool bwd) {
   if (a->d_tile < 0 || a->d_tile > kMaxDTile) return SFM_ERR_UNSUPPORTED;
   if (a->chunk < 0 || a->chunk > kMaxChunk || (a->chunk % 8) != 0) return SFM_ERR_UNSUPPORTED;
   if (a->exp2_split < 0 || a->exp2_split > 4) return SFM_ERR_UNSUPPORTED;
+  if (a->chans_per_thread < 0 || a->chans_per_thread > 2) return SFM_ERR_UNSUPPORTED;
   const void* acts[] = {a->x, a->dt, a->z, a->Bm, a->Cm, a->y};
   for (const void* p : acts)
     if (p && !aligned16(p)) return SFM_ERR_MISALIGNED;
@@ -306,6 +308,11 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
   p.d_tile = a->d_tile ? a->d_tile : v.d_tile;
   p.chunk = a->chunk ? a->chunk : v.chunk;
   p.exp2_fma_pairs = a->exp2_split ? a->exp2_split - 1 : v.exp2_pairs;
+  p.cpt = a->chans_per_thread ? a->chans_per_thread : ((a->d_tile || a->chunk) ? 1 : v.chans_per_thread);
+  // two channels per thread: the standard mixer at 8 < N <= 16 with an even tile and D
+  if (p.cpt == 2 && !(a->conv_w && a->z && a->dt_softplus && a->K == 4 && a->N > 8 && a->N <= 16 &&
+                      a->D % 2 == 0 && p.d_tile % 2 == 0))
+    p.cpt = 1;
   p.flags = (a->dt_softplus ? kSoftplus : 0) | (a->aux_init ? kAuxInit : 0) |
             (a->swap_out && a->L >= 2 ? kSwapOut : 0) | (a->conv_w ? kConv : 0) | (a->z ? kGate : 0);
   const int si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);

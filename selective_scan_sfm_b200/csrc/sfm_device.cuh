@@ -145,12 +145,42 @@ __device__ __forceinline__ void copy_span_async(char* dst, const char* base, lon
   const long long ga = g & ~15LL;
   const int total = (int)(g - ga) + cnt * esize;
   const int granules = (total + 15) >> 4;
-  for (int q = lane; q < granules; q += nlanes) {
-    const long long off = ga + 16LL * q;
-    long long rem = tensor_bytes - off;
-    const int bytes = rem >= 16 ? 16 : (rem > 0 ? (int)rem : 0);
-    cp_async16(dst + 16 * q, base + (bytes > 0 ? off : ga), bytes);
+  const char* src = base + ga;
+  if (ga + 16LL * granules <= tensor_bytes) {  // every granule lies inside the tensor
+    for (int q = lane; q < granules; q += nlanes) cp_async16(dst + 16 * q, src + 16 * q, 16);
+    return;
   }
+  for (int q = lane; q < granules; q += nlanes) {  // the span reaches the tensor's last granule
+    const long long rem = tensor_bytes - (ga + 16LL * q);
+    const int bytes = rem >= 16 ? 16 : (rem > 0 ? (int)rem : 0);
+    cp_async16(dst + 16 * q, bytes > 0 ? src + 16 * q : src, bytes);
+  }
+}
+
+// Stores the row segment staged at smem `src` (element 0 at byte (e0*esize) & 15 of a
+// 16-byte granule, the layout copy_span_async produces) to global elements
+// [e0, e0 + cnt) of `base`: 16-byte vector stores where both sides are aligned, element
+// stores at the ragged ends.  `skip0` leaves element e0 untouched.
+template <typename T>
+__device__ __forceinline__ void store_row(T* base, long long e0, const char* src_granule, int cnt, bool skip0) {
+  constexpr int es = sizeof(T), per16 = 16 / es;
+  const int head = (int)((e0 * es) & 15);
+  const T* s = reinterpret_cast<const T*>(src_granule + head);
+  T* d = base + e0;
+  int i = 0;
+  const int lead = head ? min(cnt, (16 - head) / es) : 0;  // elements before the first aligned granule
+  for (; i < lead; ++i)
+    if (!(skip0 && i == 0)) d[i] = s[i];
+  for (; i + per16 <= cnt; i += per16) {
+    const int4 v = *reinterpret_cast<const int4*>(s + i);
+    if (skip0 && i == 0) {  // only when the row starts aligned: keep element 0 as it is
+      for (int k = 1; k < per16; ++k) d[k] = s[k];
+    } else {
+      *reinterpret_cast<int4*>(d + i) = v;
+    }
+  }
+  for (; i < cnt; ++i)
+    if (!(skip0 && i == 0)) d[i] = s[i];
 }
 
 __device__ __forceinline__ int span_head(long long e0, int esize) { return (int)((e0 * esize) & 15); }

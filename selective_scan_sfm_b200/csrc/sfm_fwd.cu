@@ -38,7 +38,10 @@ namespace sfm {
 
 __device__ unsigned int g_device_error = 0;
 
-constexpr int kGroup = 4;                      // tokens per unrolled group
+#ifndef SFM_FWD_GROUP
+#define SFM_FWD_GROUP 4
+#endif
+constexpr int kGroup = SFM_FWD_GROUP;  // tokens per unrolled group
 constexpr unsigned long long kWaitNs = 2000000000ull;  // bounded wait on a bulk copy: 2 s
 
 __host__ __device__ inline int round16(int v) { return (v + 15) & ~15; }
@@ -197,6 +200,93 @@ __device__ __forceinline__ float token_out(Chan<NH>& c, const Opts& o, const flo
   return yv;
 }
 
+// CPT channels of one thread, one token: the B and C loads of the token are shared.
+template <int NH, bool RESET, int PE, int CPT>
+__device__ __forceinline__ void scan_token_multi(Chan<NH> (&c)[CPT], const float* __restrict__ bc,
+                                                 const float (&delta)[CPT], const float (&dbu)[CPT],
+                                                 float (&y)[CPT]) {
+  float2 ya[CPT], yb[CPT];
+#pragma unroll
+  for (int ch = 0; ch < CPT; ++ch) ya[ch] = yb[ch] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int k = 0; k < NH; k += (NH % 2 == 0 ? 2 : 1)) {
+    float2 Bp[2], Cp[2];
+    if constexpr (NH % 2 == 0) {
+      const float4 b4 = *reinterpret_cast<const float4*>(bc + 2 * k);
+      const float4 c4 = *reinterpret_cast<const float4*>(bc + 2 * NH + 2 * k);
+      Bp[0] = make_float2(b4.x, b4.y);
+      Bp[1] = make_float2(b4.z, b4.w);
+      Cp[0] = make_float2(c4.x, c4.y);
+      Cp[1] = make_float2(c4.z, c4.w);
+    } else {
+      Bp[0] = *reinterpret_cast<const float2*>(bc + 2 * k);
+      Cp[0] = *reinterpret_cast<const float2*>(bc + 2 * NH + 2 * k);
+    }
+#pragma unroll
+    for (int j = 0; j < (NH % 2 == 0 ? 2 : 1); ++j) {
+#pragma unroll
+      for (int ch = 0; ch < CPT; ++ch) {
+        const float2 bu = __fmul2_rn(Bp[j], make_float2(dbu[ch], dbu[ch]));
+        if constexpr (RESET) {
+          c[ch].h[k + j] = bu;
+        } else {
+          float2 a = __fmul2_rn(make_float2(delta[ch], delta[ch]), c[ch].A2[k + j]);
+          if (k + j < PE) {
+            a = exp2_fma2(a);
+          } else {
+            a.x = ex2(a.x);
+            a.y = ex2(a.y);
+          }
+          c[ch].h[k + j] = __ffma2_rn(a, c[ch].h[k + j], bu);
+        }
+        if (j == 0)
+          ya[ch] = __ffma2_rn(Cp[j], c[ch].h[k + j], ya[ch]);
+        else
+          yb[ch] = __ffma2_rn(Cp[j], c[ch].h[k + j], yb[ch]);
+      }
+    }
+  }
+#pragma unroll
+  for (int ch = 0; ch < CPT; ++ch) {
+    const float2 s2 = __fadd2_rn(ya[ch], yb[ch]);
+    y[ch] = s2.x + s2.y;
+  }
+}
+
+// CPT channels, one interior token (standard mixer path); xw[ch][0..3] are the taps.
+template <typename TI, int NH, bool STD, bool FAST, int PE, int CPT>
+__device__ __forceinline__ void token_out_multi(Chan<NH> (&c)[CPT], const Opts& o, const float* const (&xw)[CPT],
+                                                const TI (&dtv)[CPT], const TI (&zv)[CPT],
+                                                const float* __restrict__ bc, float (&yo)[CPT]) {
+  float u[CPT], delta[CPT], dbu[CPT];
+#pragma unroll
+  for (int ch = 0; ch < CPT; ++ch) {
+    if (STD || o.conv) {
+      float acc = c[ch].cb;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (STD || q < o.K) acc = fmaf(c[ch].w[q], xw[ch][q], acc);
+      u[ch] = FAST ? silu_fast(acc) : silu(acc);
+    } else {
+      u[ch] = xw[ch][0];
+    }
+    const float v = to_f(dtv[ch]) + c[ch].dtb;
+    delta[ch] = (STD || o.sp) ? (FAST ? softplus_fast(v) : softplus(v)) : v;
+    dbu[ch] = delta[ch] * u[ch];
+  }
+  float ys[CPT];
+  scan_token_multi<NH, false, PE, CPT>(c, bc, delta, dbu, ys);
+#pragma unroll
+  for (int ch = 0; ch < CPT; ++ch) {
+    float yv = fmaf(c[ch].dsk, u[ch], ys[ch]);
+    if (STD || o.gate) {
+      const float zf = to_f(zv[ch]);
+      yv *= FAST ? silu_fast(zf) : silu(zf);
+    }
+    yo[ch] = yv;
+  }
+}
+
 // xa at position s of the sample from the x row `xr` (x index q at xr[q - xlo]); aux
 // tokens are the mean; zero outside the sample or outside the staged window.
 template <typename TI>
@@ -222,36 +312,52 @@ __device__ __forceinline__ float general_token(Chan<NH>& c, const Opts& o, const
   return token_out<TI, NH, STD, false, FAST, PE>(c, o, xw, dtv, zv, bc);
 }
 
-// G interior tokens starting at chunk-relative index i: loads first (x window, dt, z),
-// then the G token computations, then the stores, so the compiler can overlap tokens.
-// xb[i + q] is the conv tap q of token i (no boundary inside the group).
-template <typename TI, typename TO, int NH, bool STD, bool FAST, int PE, int G>
-__device__ __forceinline__ void fast_group(Chan<NH>& c, const Opts& o, const TI* __restrict__ xb,
-                                           const TI* dtr, const TI* zr, TO* yr, int i,
-                                           const float* __restrict__ bct) {
+// G interior tokens of CPT channels starting at chunk-relative index i: loads first (x
+// windows, dt, z), then the token computations, then the stores, so the compiler can
+// overlap tokens and channels.  xb[ch][i + q] is conv tap q of token i of channel ch.
+template <typename TI, typename TO, int NH, bool STD, bool FAST, int PE, int G, int CPT>
+__device__ __forceinline__ void fast_group(Chan<NH> (&c)[CPT], const Opts& o, const TI* const (&xb)[CPT],
+                                           const TI* const (&dtr)[CPT], const TI* const (&zr)[CPT],
+                                           TO* const (&yr)[CPT], int i, const float* __restrict__ bct) {
   constexpr int NP2 = 4 * NH;  // floats per token in bct
-  float xv[G + 3];
+  float xv[CPT][G + 3];
+  TI dv[CPT][G], zv[CPT][G];
 #pragma unroll
-  for (int q = 0; q < G + 3; ++q) xv[q] = (q < G || STD || o.conv) ? to_f(xb[i + q]) : 0.0f;
-  TI dv[G], zv[G];
+  for (int ch = 0; ch < CPT; ++ch) {
+#pragma unroll
+    for (int q = 0; q < G + 3; ++q) xv[ch][q] = (q < G || STD || o.conv) ? to_f(xb[ch][i + q]) : 0.0f;
+#pragma unroll
+    for (int k = 0; k < G; ++k) {
+      dv[ch][k] = dtr[ch][i + k];
+      zv[ch][k] = (STD || o.gate) ? zr[ch][i + k] : dv[ch][k];
+    }
+  }
+  float yv[G][CPT];
 #pragma unroll
   for (int k = 0; k < G; ++k) {
-    dv[k] = dtr[i + k];
-    zv[k] = (STD || o.gate) ? zr[i + k] : dv[k];
+    const float* xw[CPT];
+    TI d1[CPT], z1[CPT];
+#pragma unroll
+    for (int ch = 0; ch < CPT; ++ch) {
+      xw[ch] = xv[ch] + k;
+      d1[ch] = dv[ch][k];
+      z1[ch] = zv[ch][k];
+    }
+    token_out_multi<TI, NH, STD, FAST, PE, CPT>(c, o, xw, d1, z1, bct + (i + k) * NP2, yv[k]);
   }
-  float yv[G];
 #pragma unroll
   for (int k = 0; k < G; ++k)
-    yv[k] = token_out<TI, NH, STD, false, FAST, PE>(c, o, xv + k, dv[k], zv[k], bct + (i + k) * NP2);
 #pragma unroll
-  for (int k = 0; k < G; ++k) yr[i + k] = from_f<TO>(yv[k]);
+    for (int ch = 0; ch < CPT; ++ch) yr[ch][i + k] = from_f<TO>(yv[k][ch]);
 }
 
-// Walks tokens [t0, t0 + cnt) of one sample.  xr: x row holding x indices [xlo, xhi);
-// dtr/zr/yr: rows indexed chunk-relative; bct: transposed B/C of the chunk.
-template <typename TI, typename TO, int NH, bool STD, bool FAST, int PE>
-__device__ __forceinline__ void walk(Chan<NH>& c, const Opts& o, const TI* xr, int xlo, int xhi, const TI* dtr,
-                                     const TI* zr, TO* yr, const float* bct, int t0, int cnt) {
+// Walks tokens [t0, t0 + cnt) of one sample for the thread's CPT channels.  xr[ch]: x
+// row holding x indices [xlo, xhi); dtr/zr/yr: rows indexed chunk-relative; bct:
+// transposed B/C of the chunk.  Edge tokens take the general path channel by channel.
+template <typename TI, typename TO, int NH, bool STD, bool FAST, int PE, int CPT>
+__device__ __forceinline__ void walk(Chan<NH> (&c)[CPT], const Opts& o, const TI* const (&xr)[CPT], int xlo,
+                                     int xhi, const TI* const (&dtr)[CPT], const TI* const (&zr)[CPT],
+                                     TO* const (&yr)[CPT], const float* bct, int t0, int cnt) {
   constexpr int NP2 = 4 * NH;
   // interior tokens: every conv tap on a plain x token; never the reset token
   int ta = 1, tb = 0;
@@ -264,20 +370,28 @@ __device__ __forceinline__ void walk(Chan<NH>& c, const Opts& o, const TI* xr, i
   const int e2 = max(e1, min(tend, tb));
   for (int t = t0; t < e1; ++t) {
     const int i = t - t0;
-    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD, FAST, PE>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
+#pragma unroll
+    for (int ch = 0; ch < CPT; ++ch)
+      yr[ch][i] = from_f<TO>(general_token<TI, TO, NH, STD, FAST, PE>(c[ch], o, xr[ch], xlo, xhi, t, dtr[ch][i],
+                                                                       zr[ch][i], bct + i * NP2));
   }
   if (e2 > e1) {
     // x index of tap 0 of token t is t - pl - off; xb[i + q] must be that + q
-    const TI* xb = xr + (t0 - o.pl - o.off - xlo);
+    const TI* xb[CPT];
+#pragma unroll
+    for (int ch = 0; ch < CPT; ++ch) xb[ch] = xr[ch] + (t0 - o.pl - o.off - xlo);
     int i = e1 - t0;
     const int iend = e2 - t0;
     for (; i + kGroup <= iend; i += kGroup)
-      fast_group<TI, TO, NH, STD, FAST, PE, kGroup>(c, o, xb, dtr, zr, yr, i, bct);
-    for (; i < iend; ++i) fast_group<TI, TO, NH, STD, FAST, PE, 1>(c, o, xb, dtr, zr, yr, i, bct);
+      fast_group<TI, TO, NH, STD, FAST, PE, kGroup, CPT>(c, o, xb, dtr, zr, yr, i, bct);
+    for (; i < iend; ++i) fast_group<TI, TO, NH, STD, FAST, PE, 1, CPT>(c, o, xb, dtr, zr, yr, i, bct);
   }
   for (int t = e2; t < tend; ++t) {
     const int i = t - t0;
-    yr[i] = from_f<TO>(general_token<TI, TO, NH, STD, FAST, PE>(c, o, xr, xlo, xhi, t, dtr[i], zr[i], bct + i * NP2));
+#pragma unroll
+    for (int ch = 0; ch < CPT; ++ch)
+      yr[ch][i] = from_f<TO>(general_token<TI, TO, NH, STD, FAST, PE>(c[ch], o, xr[ch], xlo, xhi, t, dtr[ch][i],
+                                                                       zr[ch][i], bct + i * NP2));
   }
 }
 
@@ -352,7 +466,8 @@ __device__ __forceinline__ Opts make_opts(const FwdParams& p) {
 // ------------------------------------------------------------------ whole-sample mode
 
 // Shared memory: [barrier 16 B][x slab][dt slab][z slab][B][C][bct][y slab if not in place]
-template <typename TI, typename TO, int NH, bool STD, int PE>
+// Thread tid owns the CPT adjacent channels CPT*tid .. CPT*tid + CPT-1 of the tile.
+template <typename TI, typename TO, int NH, bool STD, int PE, int CPT>
 __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
   constexpr bool kInPlace = std::is_same<TI, TO>::value;
   constexpr bool kFast = std::is_same<TO, __nv_bfloat16>::value;
@@ -363,8 +478,8 @@ __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
   const int d0 = blockIdx.x * p.d_tile;
   const int dcount = min(p.d_tile, p.D - d0);
   const int b1 = blockIdx.y;
-  const bool active = tid < dcount;
-  const int d = d0 + (active ? tid : 0);
+  const int c0 = tid * CPT;          // first channel of this thread within the tile
+  const bool active = c0 < dcount;   // the host keeps dcount a multiple of CPT
   const int L = p.L, N = p.N, Tx = p.Tx;
   const Opts o = make_opts(p);
   const bool swap = p.flags & kSwapOut;
@@ -386,8 +501,9 @@ __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
   }
   __syncthreads();
 
-  Chan<NH> c;
-  load_chan(c, p, d, o.conv);
+  Chan<NH> c[CPT];
+#pragma unroll
+  for (int ch = 0; ch < CPT; ++ch) load_chan(c[ch], p, d0 + (active ? c0 + ch : 0), o.conv);
 
   const unsigned xbytes = (unsigned)(dcount * Tx * si), iobytes = (unsigned)(dcount * L * si);
   const unsigned bcbytes = (unsigned)(N * L * si), ybytes = (unsigned)(dcount * L * so);
@@ -424,28 +540,40 @@ __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
     mbar_try_wait(bar, j & 1);  // completed: acquire the copied bytes in every thread
 
     transpose_bc<TI, NH>(bct, bs, cs, L * si, 0u, (unsigned)L, N, L, tid, nthr, false);
-    if (active && o.aux) c.mean = row_mean(reinterpret_cast<const TI*>(xs) + tid * Tx, Tx);
+    if (active && o.aux)
+#pragma unroll
+      for (int ch = 0; ch < CPT; ++ch) c[ch].mean = row_mean(reinterpret_cast<const TI*>(xs) + (c0 + ch) * Tx, Tx);
     __syncthreads();
 
     if (active) {
-      const TI* xr = reinterpret_cast<const TI*>(xs) + tid * Tx;
-      const TI* dtr = reinterpret_cast<const TI*>(dts) + tid * L;
-      const TI* zr = o.gate ? reinterpret_cast<const TI*>(zs) + tid * L : dtr;
-      TO* yr = kInPlace ? reinterpret_cast<TO*>(dts) + tid * L : reinterpret_cast<TO*>(ys) + tid * L;
+      const TI* xr[CPT];
+      const TI* dtr[CPT];
+      const TI* zr[CPT];
+      TO* yr[CPT];
 #pragma unroll
-      for (int k = 0; k < NH; ++k) c.h[k] = make_float2(0.f, 0.f);
-      walk<TI, TO, NH, STD, kFast, PE>(c, o, xr, 0, Tx, dtr, zr, yr, bct, 0, L);
-      if (swap) {
-        const TO h0 = yr[0];
-        yr[0] = yr[L - 1];
-        yr[L - 1] = h0;
+      for (int ch = 0; ch < CPT; ++ch) {
+        xr[ch] = reinterpret_cast<const TI*>(xs) + (c0 + ch) * Tx;
+        dtr[ch] = reinterpret_cast<const TI*>(dts) + (c0 + ch) * L;
+        zr[ch] = o.gate ? reinterpret_cast<const TI*>(zs) + (c0 + ch) * L : dtr[ch];
+        yr[ch] = kInPlace ? reinterpret_cast<TO*>(dts) + (c0 + ch) * L : reinterpret_cast<TO*>(ys) + (c0 + ch) * L;
+#pragma unroll
+        for (int k = 0; k < NH; ++k) c[ch].h[k] = make_float2(0.f, 0.f);
       }
-      if (p.final_state) {
-        float* fs = p.final_state + ((size_t)b * p.D + d) * N;
+      walk<TI, TO, NH, STD, kFast, PE, CPT>(c, o, xr, 0, Tx, dtr, zr, yr, bct, 0, L);
 #pragma unroll
-        for (int k = 0; k < NH; ++k) {
-          if (2 * k < N) fs[2 * k] = c.h[k].x;
-          if (2 * k + 1 < N) fs[2 * k + 1] = c.h[k].y;
+      for (int ch = 0; ch < CPT; ++ch) {
+        if (swap) {
+          const TO h0 = yr[ch][0];
+          yr[ch][0] = yr[ch][L - 1];
+          yr[ch][L - 1] = h0;
+        }
+        if (p.final_state) {
+          float* fs = p.final_state + ((size_t)b * p.D + d0 + c0 + ch) * N;
+#pragma unroll
+          for (int k = 0; k < NH; ++k) {
+            if (2 * k < N) fs[2 * k] = c[ch].h[k].x;
+            if (2 * k + 1 < N) fs[2 * k + 1] = c[ch].h[k].y;
+          }
         }
       }
     }
@@ -461,7 +589,11 @@ __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
 
 // ------------------------------------------------------------------ chunked mode
 
-template <typename TI, typename TO, int NH, bool STD, int PE>
+// Two staging buffers: while the threads work on step s (a chunk of one sample), the
+// copies of step s+1 (the next chunk, or the first chunk of the next sample of the folded
+// row) are in flight.  Buffer layout per stage: [x rows][dt rows][z rows][B rows][C rows];
+// after both stages: [bct][y rows if not in place].
+template <typename TI, typename TO, int NH, bool STD, int PE, int CPT>
 __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
   constexpr bool kInPlace = std::is_same<TI, TO>::value;
   constexpr bool kFast = std::is_same<TO, __nv_bfloat16>::value;
@@ -473,23 +605,25 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
   const int d0 = blockIdx.x * p.d_tile;
   const int dcount = min(p.d_tile, p.D - d0);
   const int b1 = blockIdx.y;
-  const bool active = tid < dcount;
-  const int d = d0 + (active ? tid : 0);
+  const int c0 = tid * CPT;
+  const bool active = c0 < dcount;
   const int L = p.L, N = p.N, S = p.chunk, Tx = p.Tx;
   const Opts o = make_opts(p);
   const bool swap = p.flags & kSwapOut;
   const int K = o.conv ? o.K : 1, pl = o.pl;
 
-  char* xs = smem;
-  char* dts = xs + p.d_tile * p.x_row;
-  char* zs = dts + p.d_tile * p.io_row;
-  char* bs = zs + (o.gate ? p.d_tile * p.io_row : 0);
-  char* cs = bs + N * p.io_row;
-  float* bct = reinterpret_cast<float*>(cs + N * p.io_row);
+  const int stage_bytes = p.d_tile * p.x_row + p.d_tile * p.io_row * (o.gate ? 2 : 1) + 2 * N * p.io_row;
+  float* bct = reinterpret_cast<float*>(smem + 2 * stage_bytes);
   char* ys = reinterpret_cast<char*>(bct + S * 2 * NP);
+  auto xs_of = [&](int st) { return smem + st * stage_bytes; };
+  auto dts_of = [&](int st) { return xs_of(st) + p.d_tile * p.x_row; };
+  auto zs_of = [&](int st) { return dts_of(st) + p.d_tile * p.io_row; };
+  auto bs_of = [&](int st) { return zs_of(st) + (o.gate ? p.d_tile * p.io_row : 0); };
+  auto cs_of = [&](int st) { return bs_of(st) + N * p.io_row; };
 
-  Chan<NH> c;
-  load_chan(c, p, d, o.conv);
+  Chan<NH> c[CPT];
+#pragma unroll
+  for (int ch = 0; ch < CPT; ++ch) load_chan(c[ch], p, d0 + (active ? c0 + ch : 0), o.conv);
 
   const long long x_bytes = (long long)p.B * p.D * Tx * si;
   const long long io_bytes = (long long)p.B * p.D * L * si;
@@ -501,76 +635,124 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
   const char* cg = static_cast<const char*>(p.Cm);
   TO* yg = static_cast<TO*>(p.y);
   const int nchunks = (L + S - 1) / S;
+  const int nsteps = p.B2 * nchunks;
 
-  for (int j = 0; j < p.B2; ++j) {
+  // x tokens a chunk needs: xa positions [t0-pl, t0+cnt-1+K-1-pl], clamped to the sample
+  auto x_window = [&](int t0, int cnt, int& xlo, int& xhi) {
+    const int slo = t0 - pl - o.off, shi = t0 + cnt - 1 + (K - 1 - pl) - o.off;
+    xlo = max(slo, 0);
+    xhi = min(shi + 1, Tx);
+  };
+  // issues the copies of step `st` into buffer `buf` (each thread its own rows; threads
+  // 0..2N-1 the B and C rows) and commits them as one group
+  auto stage = [&](int st, int buf) {
+    const int b = b1 * p.B2 + st / nchunks, t0 = (st % nchunks) * S, cnt = min(S, L - t0);
+    const long long row0 = (long long)b * p.D + d0;
+    int xlo, xhi;
+    x_window(t0, cnt, xlo, xhi);
+    if (active) {
+#pragma unroll
+      for (int ch = 0; ch < CPT; ++ch) {
+        const long long myrow = row0 + c0 + ch;
+        const int r = c0 + ch;
+        copy_span_async(xs_of(buf) + r * p.x_row, xg, myrow * Tx + xlo, xhi - xlo, si, x_bytes, 0, 1);
+        copy_span_async(dts_of(buf) + r * p.io_row, dtg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
+        if (o.gate) copy_span_async(zs_of(buf) + r * p.io_row, zg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
+      }
+    }
+    for (int r = tid; r < 2 * N; r += nthr) {
+      const int n = r % N;
+      const long long e0 = ((long long)b * N + n) * L + t0;
+      copy_span_async((r < N ? bs_of(buf) : cs_of(buf)) + n * p.io_row, r < N ? bg : cg, e0, cnt, si, bc_bytes, 0,
+                      1);
+    }
+    cp_async_commit();
+  };
+
+  TO head_val[CPT];
+  stage(0, 0);
+  for (int st = 0; st < nsteps; ++st) {
+    const int buf = st & 1;
+    const int j = st / nchunks, kc = st % nchunks;
     const int b = b1 * p.B2 + j;
     const long long row0 = (long long)b * p.D + d0;
-    const long long myrow = row0 + tid;
-    c.mean = (o.aux && active) ? row_mean(reinterpret_cast<const TI*>(xg) + myrow * Tx, Tx) : 0.0f;
+    const int t0 = kc * S, cnt = min(S, L - t0);
+    int xlo, xhi;
+    x_window(t0, cnt, xlo, xhi);
+    if (kc == 0) {  // a new sample: the state restarts; the aux mean needs the whole x row
 #pragma unroll
-    for (int k = 0; k < NH; ++k) c.h[k] = make_float2(0.f, 0.f);
-    TO head_val = from_f<TO>(0.0f);
-
-    for (int kc = 0; kc < nchunks; ++kc) {
-      const int t0 = kc * S, cnt = min(S, L - t0);
-      int slo = t0 - pl - o.off, shi = t0 + cnt - 1 + (K - 1 - pl) - o.off;
-      const int xlo = max(slo, 0), xhi = min(shi + 1, Tx);
-
-      // ---- stage: each thread copies its own rows; threads 0..2N-1 copy B and C rows
-      if (active) {
-        copy_span_async(xs + tid * p.x_row, xg, myrow * Tx + xlo, xhi - xlo, si, x_bytes, 0, 1);
-        copy_span_async(dts + tid * p.io_row, dtg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
-        if (o.gate) copy_span_async(zs + tid * p.io_row, zg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
+      for (int ch = 0; ch < CPT; ++ch) {
+        c[ch].mean =
+            (o.aux && active) ? row_mean(reinterpret_cast<const TI*>(xg) + (row0 + c0 + ch) * Tx, Tx) : 0.0f;
+#pragma unroll
+        for (int k = 0; k < NH; ++k) c[ch].h[k] = make_float2(0.f, 0.f);
       }
-      for (int r = tid; r < 2 * N; r += nthr) {
-        const int n = r % N;
-        const long long e0 = ((long long)b * N + n) * L + t0;
-        copy_span_async((r < N ? bs : cs) + n * p.io_row, r < N ? bg : cg, e0, cnt, si, bc_bytes, 0, 1);
-      }
-      cp_async_commit();
+    }
+    if (st + 1 < nsteps) {
+      stage(st + 1, buf ^ 1);
+      cp_async_wait<1>();  // this step's group has landed; the next one stays in flight
+    } else {
       cp_async_wait<0>();
-      __syncthreads();
+    }
+    __syncthreads();
 
-      transpose_bc<TI, NH>(bct, bs, cs, p.io_row, (unsigned)((long long)b * N * L + t0), (unsigned)L, N, cnt, tid,
-                           nthr, true);
-      __syncthreads();
+    transpose_bc<TI, NH>(bct, bs_of(buf), cs_of(buf), p.io_row, (unsigned)((long long)b * N * L + t0), (unsigned)L,
+                         N, cnt, tid, nthr, true);
+    __syncthreads();
 
-      if (active) {
-        const TI* xr = reinterpret_cast<const TI*>(xs + tid * p.x_row + span_head(myrow * Tx + xlo, si));
+    if (active) {
+      const TI* xr[CPT];
+      const TI* dtr[CPT];
+      const TI* zr[CPT];
+      TO* yr[CPT];
+#pragma unroll
+      for (int ch = 0; ch < CPT; ++ch) {
+        const long long myrow = row0 + c0 + ch;
+        const int r = c0 + ch;
+        xr[ch] = reinterpret_cast<const TI*>(xs_of(buf) + r * p.x_row + span_head(myrow * Tx + xlo, si));
         const int hd = span_head(myrow * L + t0, si);
-        const TI* dtr = reinterpret_cast<const TI*>(dts + tid * p.io_row + hd);
-        const TI* zr = o.gate ? reinterpret_cast<const TI*>(zs + tid * p.io_row + hd) : dtr;
-        TO* yr = kInPlace ? reinterpret_cast<TO*>(dts + tid * p.io_row + hd) : reinterpret_cast<TO*>(ys + tid * p.y_row);
-        walk<TI, TO, NH, STD, kFast, PE>(c, o, xr, xlo, xhi, dtr, zr, yr, bct, t0, cnt);
-        if (swap) {
-          if (t0 == 0) head_val = yr[0];  // goes to position L-1
+        dtr[ch] = reinterpret_cast<const TI*>(dts_of(buf) + r * p.io_row + hd);
+        zr[ch] = o.gate ? reinterpret_cast<const TI*>(zs_of(buf) + r * p.io_row + hd) : dtr[ch];
+        yr[ch] = kInPlace ? reinterpret_cast<TO*>(dts_of(buf) + r * p.io_row + hd)
+                          : reinterpret_cast<TO*>(ys + r * p.y_row);
+      }
+      walk<TI, TO, NH, STD, kFast, PE, CPT>(c, o, xr, xlo, xhi, dtr, zr, yr, bct, t0, cnt);
+      if (swap) {
+#pragma unroll
+        for (int ch = 0; ch < CPT; ++ch) {
+          if (t0 == 0) head_val[ch] = yr[ch][0];  // goes to position L-1
           if (t0 + cnt == L) {
-            yg[myrow * L] = yr[cnt - 1];  // the tail output becomes the next head
-            yr[cnt - 1] = head_val;
+            yg[(row0 + c0 + ch) * L] = yr[ch][cnt - 1];  // the tail output becomes the next head
+            yr[ch][cnt - 1] = head_val[ch];
           }
         }
       }
-      __syncthreads();
-
-      // ---- store the chunk's outputs, coalesced along rows
+      // in place: each thread writes its own rows back, 16-byte stores where aligned
+      if (kInPlace)
+#pragma unroll
+        for (int ch = 0; ch < CPT; ++ch)
+          store_row<TO>(yg, (row0 + c0 + ch) * L + t0, dts_of(buf) + (c0 + ch) * p.io_row, cnt, swap && t0 == 0);
+      if (p.final_state && kc == nchunks - 1) {
+#pragma unroll
+        for (int ch = 0; ch < CPT; ++ch) {
+          float* fs = p.final_state + ((size_t)b * p.D + d0 + c0 + ch) * N;
+#pragma unroll
+          for (int k = 0; k < NH; ++k) {
+            if (2 * k < N) fs[2 * k] = c[ch].h[k].x;
+            if (2 * k + 1 < N) fs[2 * k + 1] = c[ch].h[k].y;
+          }
+        }
+      }
+    }
+    __syncthreads();  // the buffer of this step is free for the copies of step st + 2
+    if (!kInPlace) {  // separate output rows: coalesced element stores by rows
       for (int r = warp; r < dcount; r += nwarps) {
-        const long long rr = row0 + r;
-        const char* src = kInPlace ? dts + r * p.io_row + span_head(rr * L + t0, si) : ys + r * p.y_row;
-        TO* dst = yg + rr * L + t0;
+        const char* src = ys + r * p.y_row;
+        TO* dst = yg + (row0 + r) * L + t0;
         for (int i = lane; i < cnt; i += 32)
           if (!(swap && t0 + i == 0)) dst[i] = *reinterpret_cast<const TO*>(src + i * so);
       }
-      // the next chunk's copies overwrite the staged rows only after every thread has
-      // passed the __syncthreads that follows them, i.e. after this loop
-    }
-
-    if (p.final_state && active) {
-      float* fs = p.final_state + ((size_t)b * p.D + d) * N;
-#pragma unroll
-      for (int k = 0; k < NH; ++k) {
-        if (2 * k < N) fs[2 * k] = c.h[k].x;
-        if (2 * k + 1 < N) fs[2 * k + 1] = c.h[k].y;
-      }
+      __syncthreads();  // ys is rewritten by the next step's walk
     }
   }
 }
@@ -838,6 +1020,7 @@ int fwd_chunk_smem(const FwdParams& p, int si, int so, int NP) {
   s += (long long)p.d_tile * p.x_row;
   s += (long long)p.d_tile * p.io_row * (gate ? 2 : 1);
   s += 2LL * p.N * p.io_row;
+  s *= 2;  // two staging buffers
   s += (long long)p.chunk * 2 * NP * 4;
   if (si != so) s += (long long)p.d_tile * p.y_row;
   return s > (1LL << 30) ? (1 << 30) : (int)s;
@@ -881,20 +1064,29 @@ static cudaError_t launch_lanes(const FwdParams& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <typename TI, typename TO, int NH, bool STD, int PE>
-static cudaError_t launch_t(const FwdParams& p, cudaStream_t s) {
+template <typename TI, typename TO, int NH, bool STD, int PE, int CPT>
+static cudaError_t launch_cpt(const FwdParams& p, cudaStream_t s) {
   static int whole_set = 48 * 1024, chunk_set = 48 * 1024;
-  const int threads = (p.d_tile + 31) & ~31;
+  const int threads = ((p.d_tile + CPT - 1) / CPT + 31) & ~31;
   dim3 grid((p.D + p.d_tile - 1) / p.d_tile, p.B / p.B2);
   cudaError_t e;
   if (p.mode == kModeWhole) {
-    if ((e = set_smem(fwd_whole_kernel<TI, TO, NH, STD, PE>, p.smem_bytes, whole_set)) != cudaSuccess) return e;
-    fwd_whole_kernel<TI, TO, NH, STD, PE><<<grid, threads, p.smem_bytes, s>>>(p);
+    if ((e = set_smem(fwd_whole_kernel<TI, TO, NH, STD, PE, CPT>, p.smem_bytes, whole_set)) != cudaSuccess) return e;
+    fwd_whole_kernel<TI, TO, NH, STD, PE, CPT><<<grid, threads, p.smem_bytes, s>>>(p);
   } else {
-    if ((e = set_smem(fwd_chunk_kernel<TI, TO, NH, STD, PE>, p.smem_bytes, chunk_set)) != cudaSuccess) return e;
-    fwd_chunk_kernel<TI, TO, NH, STD, PE><<<grid, threads, p.smem_bytes, s>>>(p);
+    if ((e = set_smem(fwd_chunk_kernel<TI, TO, NH, STD, PE, CPT>, p.smem_bytes, chunk_set)) != cudaSuccess) return e;
+    fwd_chunk_kernel<TI, TO, NH, STD, PE, CPT><<<grid, threads, p.smem_bytes, s>>>(p);
   }
   return cudaGetLastError();
+}
+
+// Two channels per thread are built for the standard mixer at N = 16 only.
+template <typename TI, typename TO, int NH, bool STD, int PE>
+static cudaError_t launch_t(const FwdParams& p, cudaStream_t s) {
+  if constexpr (STD && NH == 8) {
+    if (p.cpt == 2) return launch_cpt<TI, TO, NH, STD, PE, 2>(p, s);
+  }
+  return launch_cpt<TI, TO, NH, STD, PE, 1>(p, s);
 }
 
 // The standard mixer (conv K=4 + softplus + gate) gets the specialised path and, at

@@ -39,27 +39,32 @@ def divisors_upto(B, cap):
     return [v for v in (1, 2, 4, 8, 16, 32) if v <= cap and B % v == 0]
 
 
-def candidates(B, T, D):
-    """(B2, d_tile, chunk, lanes): one thread per channel (lanes = 1) with whole-sample or
-    chunked staging, and, for longer samples, P lanes per channel (chunk = 8 P)."""
+def candidates(B, T, D, N=16):
+    """(B2, d_tile, chunk, lanes, chans_per_thread): one thread per channel or two side by
+    side (lanes = 1) with whole-sample or chunked staging, and, for longer samples, P lanes
+    per channel (chunk = 8 P)."""
     L = T + 2
     out = []
     tiles = [t for t in (32, 64, 128) if t <= max(32, ((D + 31) // 32) * 32)]
     chunks = sorted(set([c for c in (32, 56, 64, 128) if c < L] + [((L + 7) // 8) * 8 if L <= 256 else 0]) - {0})
-    for B2, dt, ch in itertools.product(divisors_upto(B, 32), tiles, chunks):
-        out.append((B2, dt, ch, 1))
+    cpts = (1, 2) if (8 < N <= 16 and D % 2 == 0) else (1,)
+    for B2, dt, ch, cpt in itertools.product(divisors_upto(B, 32), tiles, chunks, cpts):
+        if cpt == 2 and B2 > 4:
+            continue
+        out.append((B2, dt, ch, 1, cpt))
     if L >= 100:
         for B2, P, threads in itertools.product(divisors_upto(B, 4), (2, 4, 8, 16, 32), (64, 128, 256)):
             if threads // P >= 1 and 8 * P <= 4 * L:
-                out.append((B2, threads // P, 8 * P, P))
+                out.append((B2, threads // P, 8 * P, P, 1))
     return out
 
 
-def time_variant(sets, lib, stream, B2, d_tile, chunk, reps, exp2_split=0, lanes=1):
+def time_variant(sets, lib, stream, B2, d_tile, chunk, reps, exp2_split=0, lanes=1, cpt=1):
     args = []
     for s in sets:
         a = s["args"]
         a.B1, a.d_tile, a.chunk, a.exp2_split, a.lanes = s["B"] // B2, d_tile, chunk, exp2_split, lanes
+        a.chans_per_thread = cpt
         args.append(ctypes.byref(a))
     sp = ctypes.c_void_p(stream.cuda_stream)
     for i in range(3):
@@ -98,17 +103,17 @@ def sweep(grid, reps=15, log=print):
             sets.append(dict(args=a, keep=(dc, y), B=B))
         rows = []
         split0 = 3 if N == 16 else 1  # stage 1 at two FMA-pipe exp2 pairs (N = 16)
-        for (B2, dtile, ch, P) in candidates(B, T, D):
-            ms = time_variant(sets, lib, stream, B2, dtile, ch, reps, split0, P)
+        for (B2, dtile, ch, P, cpt) in candidates(B, T, D, N):
+            ms = time_variant(sets, lib, stream, B2, dtile, ch, reps, split0, P, cpt)
             if ms is None:
                 continue
-            rows.append(dict(B2=B2, d_tile=dtile, chunk=ch, lanes=P, exp2_pairs=split0 - 1, ms=ms,
+            rows.append(dict(B2=B2, d_tile=dtile, chunk=ch, lanes=P, cpt=cpt, exp2_pairs=split0 - 1, ms=ms,
                              gelem_s=B * D * (T + 2) / ms / 1e6))
         rows.sort(key=lambda r: r["ms"])
         if N == 16 and rows[0]["lanes"] == 1:  # stage 2: the exp2 split for the best launch shape
             b0 = rows[0]
             for split in (1, 2, 4):
-                ms = time_variant(sets, lib, stream, b0["B2"], b0["d_tile"], b0["chunk"], reps, split, 1)
+                ms = time_variant(sets, lib, stream, b0["B2"], b0["d_tile"], b0["chunk"], reps, split, 1, b0["cpt"])
                 if ms is not None:
                     rows.append(dict(b0, exp2_pairs=split - 1, ms=ms, gelem_s=B * D * (T + 2) / ms / 1e6))
             rows.sort(key=lambda r: r["ms"])
@@ -116,10 +121,10 @@ def sweep(grid, reps=15, log=print):
         unfolded = min((r for r in rows if r["B2"] == 1), key=lambda r: r["ms"])
         res = dict(T=T, B=B, D=D, N=N, dtype=dtype, best=best, best_unfolded=unfolded, all=rows)
         results.append(res)
-        log("T=%4d B=%4d D=%5d N=%2d best B2=%2d lanes=%2d d_tile=%3d chunk=%3d exp2_pairs=%d %.4f ms "
+        log("T=%4d B=%4d D=%5d N=%2d best B2=%2d lanes=%2d cpt=%d d_tile=%3d chunk=%3d exp2_pairs=%d %.4f ms "
             "(%.1f Gelem/s); best unfolded %.4f ms -> folding speedup %.3f" % (
-                T, B, D, N, best["B2"], best["lanes"], best["d_tile"], best["chunk"], best["exp2_pairs"], best["ms"],
-                best["gelem_s"], unfolded["ms"], unfolded["ms"] / best["ms"]))
+                T, B, D, N, best["B2"], best["lanes"], best["cpt"], best["d_tile"], best["chunk"], best["exp2_pairs"],
+                best["ms"], best["gelem_s"], unfolded["ms"], unfolded["ms"] / best["ms"]))
         del sets
         torch.cuda.empty_cache()
     return results
@@ -130,11 +135,12 @@ def write_lut(results, path=LUT, gpu=None):
     lines = ["// sfm_lut.inc -- adaptive-B1 look-up table: launch choices measured on B200.",
              "// Written by selective_scan_sfm_b200/lut_sweep.py from a sweep over B, T, D and N on %s;" % gpu,
              "// each row is the fastest measured variant for that shape.",
-             "// Columns: T, B, D, N, B2, lanes, d_tile, chunk, exp2_pairs."]
+             "// Columns: T, B, D, N, B2, lanes, d_tile, chunk, exp2_pairs, chans_per_thread."]
     for r in results:
         b = r["best"]
-        lines.append("{%d, %d, %d, %d, %d, %d, %d, %d, %d}," % (r["T"], r["B"], r["D"], r["N"], b["B2"], b["lanes"],
-                                                               b["d_tile"], b["chunk"], b["exp2_pairs"]))
+        lines.append("{%d, %d, %d, %d, %d, %d, %d, %d, %d, %d}," % (
+            r["T"], r["B"], r["D"], r["N"], b["B2"], b["lanes"], b["d_tile"], b["chunk"], b["exp2_pairs"],
+            b.get("cpt", 1)))
     open(path, "w").write("\n".join(lines) + "\n")
 
 

@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.sfm_abi_version() == 2
+    assert L.sfm_abi_version() == 3
     for code in range(6):
         assert _abi.status_string(code).startswith("SFM_")
     assert _abi.status_string(99) == "SFM_ERR_UNKNOWN"

@@ -269,3 +269,28 @@ def test_lanes_sample_isolation():
         p[field][1] = float("nan")
         y1 = fused(p, lanes=8, d_tile=16, B1=1)
         assert torch.equal(y1[[0, 2, 3]], y0[[0, 2, 3]]), field
+
+
+# ------------------------------------------------------------------ two channels per thread
+
+CPT2_GRID = [
+    # B, D, T, N, dtype, d_tile, chunk (chunk >= L: whole-sample staging)
+    (4, 128, 49, 16, "bf16", 64, 56),
+    (3, 70, 49, 12, "f32", 32, 56),
+    (2, 96, 120, 16, "bf16", 64, 32),
+    (2, 34, 75, 16, "f32", 32, 24),
+]
+
+
+@pytest.mark.parametrize("B,D,T,N,dtype,d_tile,chunk", CPT2_GRID)
+def test_two_channels_per_thread(B, D, T, N, dtype, d_tile, chunk):
+    d = synth.make_inputs(B=B, D=D, T=T, N=N, dtype=dtype, seed=8000 + D + T, random_A=True)
+    dc = to_cuda(d)
+    for swap in (False, True):
+        fs = torch.full((B, D, N), float("nan"), device="cuda")
+        y = fused(dc, swap_out=swap, d_tile=d_tile, chunk=chunk, chans_per_thread=2, B1=B, final_state=fs)
+        ref, ref_state = oracle_layer(d, swap_out=swap, want_state=True)
+        check(y, ref, dtype, "cpt=2 swap=%s" % swap)
+        assert rel_err(fs.double().cpu().numpy(), ref_state) <= TOL[dtype]
+        y1 = fused(dc, swap_out=swap, d_tile=d_tile, chunk=chunk, chans_per_thread=1, B1=B)
+        assert rel_err(y.double().cpu().numpy(), y1.double().cpu().numpy()) <= TOL[dtype]
