@@ -46,7 +46,7 @@ def candidates(B, T, D, N=16):
     L = T + 2
     out = []
     tiles = [t for t in (32, 64, 128) if t <= max(32, ((D + 31) // 32) * 32)]
-    chunks = sorted(set([c for c in (32, 56, 64, 128) if c < L] + [((L + 7) // 8) * 8 if L <= 256 else 0]) - {0})
+    chunks = sorted(set([c for c in (16, 24, 32, 56, 64, 128) if c < L] + [((L + 7) // 8) * 8 if L <= 256 else 0]) - {0})
     cpts = (1, 2) if (8 < N <= 16 and D % 2 == 0) else (1,)
     for B2, dt, ch, cpt in itertools.product(divisors_upto(B, 32), tiles, chunks, cpts):
         if cpt == 2 and B2 > 4:
