@@ -60,7 +60,10 @@ def _load():
         lib.ora_scan.argtypes = scan_args + [_l, _l]
         lib.ora_scan_folded.argtypes = scan_args + [_l]
         lib.ora_scan_bwd.argtypes = [_dp] * 17 + [_l, _l, _l, _l, _i]
-        for f in ("ora_aux_init", "ora_aux_swap", "ora_conv1d", "ora_scan", "ora_scan_folded", "ora_scan_bwd"):
+        lib.ora_conv1d_bwd.argtypes = [_dp] * 7 + [_l, _l, _l, _i, _i, _i]
+        lib.ora_aux_init_bwd.argtypes = [_dp, _dp, _l, _l, _l]
+        for f in ("ora_aux_init", "ora_aux_swap", "ora_conv1d", "ora_scan", "ora_scan_folded", "ora_scan_bwd",
+                  "ora_conv1d_bwd", "ora_aux_init_bwd"):
             getattr(lib, f).restype = None
         _lib = lib
     return _lib
@@ -208,3 +211,44 @@ def mixer_layer(x, dt, z, Bm, Cm, A, Dskip, dt_bias, conv_w, conv_b, *, aux_init
     if swap_out:
         y = aux_swap(y)
     return (y, fs) if want_state else y
+
+
+def conv1d_bwd(xa, w, bias, du, pad_left=None, silu=True):
+    """Gradients of conv1d(+SiLU) w.r.t. its input, weights and bias, given dLoss/du."""
+    xa, w, bias, du = _f64(xa), _f64(w), _f64(bias), _f64(du)
+    B, D, L = xa.shape
+    K = w.shape[1]
+    pad_left = (K - 1) // 2 if pad_left is None else pad_left
+    dxa = np.empty_like(xa)
+    dw = np.zeros((D, K))
+    db = np.zeros(D) if bias is not None else None
+    _load().ora_conv1d_bwd(_p(xa), _p(w), _p(bias), _p(du), _p(dxa), _p(dw), _p(db), B, D, L, K, pad_left, int(silu))
+    return dxa, dw, db
+
+
+def aux_init_bwd(dxa):
+    """dLoss/dx from dLoss/dxa for xa = [mean(x), x, mean(x)]."""
+    dxa = _f64(dxa)
+    B, D, L = dxa.shape
+    dx = np.empty((B, D, L - 2))
+    _load().ora_aux_init_bwd(_p(dxa), _p(dx), B, D, L - 2)
+    return dx
+
+
+def mixer_layer_bwd(x, dt, z, Bm, Cm, A, Dskip, dt_bias, conv_w, conv_b, dout, *, aux_init_in=False,
+                    swap_out=False, pad_left=None, dt_softplus=True):
+    """Gradients of mixer_layer's output w.r.t. every input and parameter, composed from
+    the single-step backwards in reverse order: swap, gate + scan, SiLU + conv, aux init."""
+    dout = _f64(dout)
+    if swap_out:
+        dout = aux_swap(dout)  # the swap is its own inverse
+    xa = aux_init(x) if aux_init_in else _f64(x)
+    K = conv_w.shape[1]
+    u = conv1d(xa, conv_w, conv_b, K=K, pad_left=pad_left, silu=True)
+    g = scan_bwd(u, dt, Bm, Cm, A, dout, Dskip, dt_bias, z, dt_softplus)
+    dxa, dw, db = conv1d_bwd(xa, conv_w, conv_b, g.pop("du"), pad_left=pad_left, silu=True)
+    g["dx"] = aux_init_bwd(dxa) if aux_init_in else dxa
+    g["dconv_w"] = dw
+    if db is not None:
+        g["dconv_b"] = db
+    return g

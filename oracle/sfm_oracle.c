@@ -269,3 +269,62 @@ void ora_scan_bwd(const double* u, const double* dt, const double* z,
     }
   free(h); free(abar); free(delta); free(g);
 }
+
+/* Backward of ora_conv1d (+ SiLU when silu != 0) given du = dLoss/du:
+ *   pre = bias + sum_k w[k] * xa[t+k-pad_left] (zero outside the sample), u = act(pre);
+ *   dpre[t] = du[t] * act'(pre[t]);  dxa[s] = sum_k w[k] * dpre[s-k+pad_left] (inside the sample);
+ *   dw[d,k] = sum_{b,t} dpre[b,d,t] * xa[b,d,t+k-pad_left];  dbias[d] = sum_{b,t} dpre[b,d,t].
+ * dw and dbias (if not NULL) are zeroed and accumulated. */
+void ora_conv1d_bwd(const double* xa, const double* w, const double* bias, const double* du,
+                    double* dxa, double* dw, double* dbias,
+                    long B, long D, long L, int K, int pad_left, int silu) {
+  double* dpre = (double*)malloc(sizeof(double) * (size_t)L);
+  memset(dw, 0, sizeof(double) * (size_t)(D * K));
+  if (dbias) memset(dbias, 0, sizeof(double) * (size_t)D);
+  for (long b = 0; b < B; ++b)
+    for (long d = 0; d < D; ++d) {
+      const double* xr = xa + (b * D + d) * L;
+      const double* dur = du + (b * D + d) * L;
+      double* dxr = dxa + (b * D + d) * L;
+      for (long t = 0; t < L; ++t) {
+        double pre = bias ? bias[d] : 0.0;
+        for (int k = 0; k < K; ++k) {
+          const long s = t + k - pad_left;
+          if (s >= 0 && s < L) pre += w[d * K + k] * xr[s];
+        }
+        double g = 1.0;
+        if (silu) {
+          const double sg = ora_sigmoid(pre);
+          g = sg * (1.0 + pre * (1.0 - sg));
+        }
+        dpre[t] = dur[t] * g;
+      }
+      for (long s = 0; s < L; ++s) {
+        double acc = 0.0;
+        for (int k = 0; k < K; ++k) {
+          const long t = s - k + pad_left;
+          if (t >= 0 && t < L) acc += w[d * K + k] * dpre[t];
+        }
+        dxr[s] = acc;
+      }
+      for (long t = 0; t < L; ++t) {
+        for (int k = 0; k < K; ++k) {
+          const long s = t + k - pad_left;
+          if (s >= 0 && s < L) dw[d * K + k] += dpre[t] * xr[s];
+        }
+        if (dbias) dbias[d] += dpre[t];
+      }
+    }
+  free(dpre);
+}
+
+/* Backward of ora_aux_init: xa = [m, x_0..x_{T-1}, m] with m the mean of x, so
+ * dx[t] = dxa[t+1] + (dxa[0] + dxa[T+1]) / T. */
+void ora_aux_init_bwd(const double* dxa, double* dx, long B, long D, long T) {
+  const long L = T + 2;
+  for (long r = 0; r < B * D; ++r) {
+    const double* g = dxa + r * L;
+    const double share = (g[0] + g[L - 1]) / (double)T;
+    for (long t = 0; t < T; ++t) dx[r * T + t] = g[t + 1] + share;
+  }
+}

@@ -23,6 +23,8 @@ MUTATIONS = {
     "bwd_dA_missing_delta": ("dA[d * N + n] += da * abar[t * N + n] * delta[t];", "dA[d * N + n] += da * abar[t * N + n];"),
     "softplus_threshold": ("return v > 20.0 ? v : log1p(exp(v));", "return v > 2.0 ? v : log1p(exp(v));"),
     "swap_keeps_head": ("yr[0] = yr[L - 1];", "yr[0] = yr[0];"),
+    "conv_bwd_index": ("const long t = s - k + pad_left;", "const long t = s + k - pad_left;"),
+    "aux_bwd_no_mean_share": ("const double share = (g[0] + g[L - 1]) / (double)T;", "const double share = 0.0;"),
 }
 
 

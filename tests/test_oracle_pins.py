@@ -378,3 +378,75 @@ def test_threads_do_not_change_results(ora):
     y1 = ora.scan(c["u"], c["dt"], c["Bm"], c["Cm"], c["A"], c["Dskip"], c["dt_bias"], c["z"], threads=1)
     y4 = ora.scan(c["u"], c["dt"], c["Bm"], c["Cm"], c["A"], c["Dskip"], c["dt_bias"], c["z"], threads=4)
     np.testing.assert_array_equal(y1, y4)
+
+
+# ---------------------------------------------------------------- the mixer layer backward
+
+def test_conv_and_aux_backward_are_adjoints(ora):
+    """For the linear parts, <f(a), v> = <a, f^T(v)>: conv without bias/SiLU and aux init."""
+    B, D, L, K = 2, 3, 9, 4
+    xa, w, v = rnd((B, D, L), 100), rnd((D, K), 101), rnd((B, D, L), 102)
+    for pl in (0, 1, 3):
+        u = ora.conv1d(xa, w, None, K=K, pad_left=pl, silu=False)
+        dxa, dw, _ = ora.conv1d_bwd(xa, w, None, v, pad_left=pl, silu=False)
+        assert float((u * v).sum()) == pytest.approx(float((xa * dxa).sum()), rel=1e-12)
+        # dw from the library conv's autograd
+        t = torch.tensor(xa, requires_grad=False)
+        wt = torch.tensor(w, requires_grad=True)
+        out = torch.nn.functional.conv1d(torch.nn.functional.pad(t, (pl, K - 1 - pl)), wt.unsqueeze(1), groups=D)
+        (out * torch.from_numpy(v)).sum().backward()
+        np.testing.assert_allclose(dw, wt.grad.numpy(), rtol=1e-12, atol=1e-13)
+    x, g = rnd((B, D, 7), 103), rnd((B, D, 9), 104)
+    assert float((ora.aux_init(x) * g).sum()) == pytest.approx(float((x * ora.aux_init_bwd(g)).sum()), rel=1e-12)
+
+
+def _mixer_loss(ora, p, dout, aux, swap):
+    y = ora.mixer_layer(p["x"], p["dt"], p["z"], p["Bm"], p["Cm"], p["A"], p["Dskip"], p["dt_bias"], p["conv_w"],
+                        p["conv_b"], aux_init_in=aux, swap_out=swap)
+    return float((y * dout).sum())
+
+
+@pytest.mark.parametrize("aux,swap", [(True, True), (False, False)])
+def test_mixer_backward_finite_differences(ora, aux, swap):
+    d = synth.make_inputs(B=2, D=2, T=5, N=2, dtype="f32", seed=110, aux=aux, random_A=True)
+    p = {k: d[k].double().numpy().copy() for k in ("x", "dt", "z", "Bm", "Cm", "A", "Dskip", "dt_bias",
+                                                   "conv_w", "conv_b")}
+    L = p["dt"].shape[-1]
+    dout = rnd((2, 2, L), 111)
+    g = ora.mixer_layer_bwd(p["x"], p["dt"], p["z"], p["Bm"], p["Cm"], p["A"], p["Dskip"], p["dt_bias"],
+                            p["conv_w"], p["conv_b"], dout, aux_init_in=aux, swap_out=swap)
+    names = {"x": "dx", "conv_w": "dconv_w", "conv_b": "dconv_b", "dt": "ddt", "z": "dz", "Bm": "dB",
+             "A": "dA", "dt_bias": "ddt_bias"}
+    h = 1e-6
+    for f, gname in names.items():
+        arr = p[f]
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            keep = arr[idx]
+            arr[idx] = keep + h; lp = _mixer_loss(ora, p, dout, aux, swap)
+            arr[idx] = keep - h; lm = _mixer_loss(ora, p, dout, aux, swap)
+            arr[idx] = keep
+            num[idx] = (lp - lm) / (2 * h)
+        np.testing.assert_allclose(g[gname], num, rtol=2e-6, atol=2e-8, err_msg=gname)
+
+
+def test_mixer_backward_matches_autograd_of_library_composition(ora):
+    d = synth.make_inputs(B=3, D=4, T=11, N=4, dtype="f32", seed=120, random_A=True)
+    names = ("x", "dt", "z", "Bm", "Cm", "A", "Dskip", "dt_bias", "conv_w", "conv_b")
+    p = {k: d[k].double().numpy() for k in names}
+    dout = rnd((3, 4, 13), 121)
+    g = ora.mixer_layer_bwd(p["x"], p["dt"], p["z"], p["Bm"], p["Cm"], p["A"], p["Dskip"], p["dt_bias"],
+                            p["conv_w"], p["conv_b"], dout, aux_init_in=True, swap_out=True)
+    T = {k: torch.tensor(v, requires_grad=True) for k, v in p.items()}
+    xt = T["x"]
+    m = xt.mean(-1, keepdim=True)
+    xa = torch.cat([m, xt, m], -1)
+    u = torch.nn.functional.silu(torch.nn.functional.conv1d(
+        torch.nn.functional.pad(xa, (1, 2)), T["conv_w"].unsqueeze(1), T["conv_b"], groups=4))
+    y = materialised(u, T["dt"], T["z"], T["Bm"], T["Cm"], T["A"], T["Dskip"], T["dt_bias"], lib=torch)
+    y = torch.cat([y[..., -1:], y[..., 1:-1], y[..., :1]], -1)  # swap
+    (y * torch.from_numpy(dout)).sum().backward()
+    pairs = {"x": "dx", "conv_w": "dconv_w", "conv_b": "dconv_b", "dt": "ddt", "z": "dz", "Bm": "dB", "Cm": "dC",
+             "A": "dA", "Dskip": "dDskip", "dt_bias": "ddt_bias"}
+    for f, gname in pairs.items():
+        np.testing.assert_allclose(g[gname], T[f].grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=gname)
