@@ -241,6 +241,39 @@ SFM_API sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* args
                                                        const sfm_scan_grads* grads,
                                                        sfm_stream_t stream);
 
+/* Gradients of the whole mixer layer (all fp32, caller-owned device memory). */
+typedef struct {
+  uint32_t size;        /* sizeof(sfm_mixer_grads)                                    */
+  const void* dout;     /* [B,D,L] gradient of the layer output y as the forward stored
+                           it (after the swap when swap_out), args->out_dtype          */
+  float* dx;            /* [B,D,L-2] if aux_init else [B,D,L]: gradient of x          */
+  float* dconv_w;       /* [D,K] (required when args->conv_w is given)                */
+  float* dconv_b;       /* [D] or NULL when args->conv_b is NULL                      */
+  float* ddt;           /* [B,D,L]                                                    */
+  float* dz;            /* [B,D,L] or NULL when args->z is NULL                       */
+  float* dA;            /* [D,N]                                                      */
+  float* dDskip;        /* [D] or NULL when args->Dskip is NULL                       */
+  float* ddt_bias;      /* [D] or NULL when args->dt_bias is NULL                     */
+  float* dB;            /* [B,N,L]                                                    */
+  float* dC;            /* [B,N,L]                                                    */
+} sfm_mixer_grads;
+
+/* Workspace (bytes, 256-byte aligned device memory) sfm_mixer_bwd needs for `args`. */
+SFM_API sfm_status sfm_mixer_bwd_workspace_size(const sfm_scan_args* args, size_t* bytes);
+
+/*
+ * Backward of the whole fused layer of sfm_selective_scan_fold -- aux init, conv +
+ * SiLU, Delta, folded scan, D skip, gate and swap -- for the same args (y is not read):
+ * the output gradient is read through the swap, the scan input is rebuilt from x, the
+ * scan backward runs as in sfm_selective_scan_fold_bwd, then the conv + SiLU backward
+ * gives dx (plus the aux mean's share (dxa[0] + dxa[L-1]) / T on every token when
+ * aux_init), dconv_w and dconv_b.  Every reduction runs in a fixed order (bitwise
+ * reproducible).  Overwrites every gradient buffer given.  Sources: the layer as
+ * defined at the top of this header; the backward itself is not on the pages.
+ */
+SFM_API sfm_status sfm_mixer_bwd(const sfm_scan_args* args, const sfm_mixer_grads* grads, void* workspace,
+                                 size_t workspace_bytes, sfm_stream_t stream);
+
 /*
  * Adaptive B1: the number of folded rows for a batch of B samples of T patch tokens,
  * D channels and state size N, from a look-up table built by a B200 sweep.  The

@@ -16,7 +16,7 @@ from ._abi import SFM_BF16, SFM_F32, SfmError
 
 __all__ = [
     "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d", "sfm_selective_scan_fold",
-    "sfm_selective_scan_fold_bwd", "sfm_selective_scan_fold_bwd_noalloc", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
+    "sfm_selective_scan_fold_bwd", "sfm_selective_scan_fold_bwd_noalloc", "sfm_mixer_bwd", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
     "SfmError", "library_path",
 ]
 
@@ -208,6 +208,45 @@ def sfm_selective_scan_fold_bwd_noalloc(u, dt, Bm, Cm, A, dout, grads, *, z=None
         setattr(g, k, None if t is None else _dev(t, k, torch.float32).data_ptr())
     _abi.check(_abi.lib().sfm_selective_scan_fold_bwd_noalloc(ctypes.byref(a), ctypes.byref(g), _stream(stream)),
                "sfm_selective_scan_fold_bwd_noalloc")
+    return grads
+
+
+def sfm_mixer_bwd(x, dt, Bm, Cm, A, dout, *, z=None, Dskip=None, dt_bias=None, conv_w=None, conv_b=None,
+                  pad_left=None, dt_softplus=True, aux_init=False, swap_out=False, workspace=None, stream=None):
+    """Backward of the whole fused layer (same arguments as sfm_selective_scan_fold).
+    dout is the gradient of the stored output (after the swap).  Returns fp32 grads:
+    dx, dconv_w, dconv_b, ddt, dz, dA, dDskip, ddt_bias, dB, dC (those that apply)."""
+    a, _ = _scan_args(x, dt, Bm, Cm, A, z, Dskip, dt_bias, conv_w, conv_b, None, None, 0, pad_left, dt_softplus,
+                      aux_init, swap_out, None, 0, 0, 0, need_y=False)
+    B, D, L, N = a.B, a.D, a.L, a.N
+    _dev(dout, "dout", dt.dtype, (B, D, L))
+    dev, f32 = dt.device, torch.float32
+    e = lambda *shape: torch.empty(*shape, dtype=f32, device=dev)
+    grads = dict(dx=e(*x.shape), ddt=e(B, D, L), dA=e(D, N), dB=e(B, N, L), dC=e(B, N, L))
+    if conv_w is not None:
+        grads["dconv_w"] = e(*conv_w.shape)
+        if conv_b is not None:
+            grads["dconv_b"] = e(D)
+    if z is not None:
+        grads["dz"] = e(B, D, L)
+    if Dskip is not None:
+        grads["dDskip"] = e(D)
+    if dt_bias is not None:
+        grads["ddt_bias"] = e(D)
+    g = _abi.MixerGrads()
+    g.size = ctypes.sizeof(_abi.MixerGrads)
+    g.dout = dout.data_ptr()
+    for k in ("dx", "dconv_w", "dconv_b", "ddt", "dz", "dA", "dDskip", "ddt_bias", "dB", "dC"):
+        t = grads.get(k)
+        setattr(g, k, None if t is None else t.data_ptr())
+    need = ctypes.c_size_t(0)
+    _abi.check(_abi.lib().sfm_mixer_bwd_workspace_size(ctypes.byref(a), ctypes.byref(need)),
+               "sfm_mixer_bwd_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(max(int(need.value), 1), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8)
+    _abi.check(_abi.lib().sfm_mixer_bwd(ctypes.byref(a), ctypes.byref(g), ctypes.c_void_p(workspace.data_ptr()),
+                                        workspace.numel(), _stream(stream)), "sfm_mixer_bwd")
     return grads
 
 

@@ -19,6 +19,7 @@ ENTRY_POINTS = (
     "sfm_status_string", "sfm_abi_version", "sfm_last_cuda_error", "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d",
     "sfm_selective_scan_fold", "sfm_scan_bwd_workspace_size", "sfm_selective_scan_fold_bwd",
     "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error", "sfm_selective_scan_fold_bwd_noalloc",
+    "sfm_mixer_bwd_workspace_size", "sfm_mixer_bwd",
 )
 
 #: Size of the workspace built into the library for sfm_selective_scan_fold_bwd_noalloc.
@@ -50,6 +51,15 @@ class ScanGrads(ctypes.Structure):
         ("size", ctypes.c_uint32),
         ("dout", _vp), ("du", _vp), ("ddt", _vp), ("dz", _vp), ("dA", _vp),
         ("dDskip", _vp), ("ddt_bias", _vp), ("dB", _vp), ("dC", _vp),
+    ]
+
+
+class MixerGrads(ctypes.Structure):
+    """Mirror of sfm_mixer_grads."""
+    _fields_ = [
+        ("size", ctypes.c_uint32),
+        ("dout", _vp), ("dx", _vp), ("dconv_w", _vp), ("dconv_b", _vp), ("ddt", _vp), ("dz", _vp),
+        ("dA", _vp), ("dDskip", _vp), ("ddt_bias", _vp), ("dB", _vp), ("dC", _vp),
     ]
 
 
@@ -87,6 +97,8 @@ def lib():
         L.sfm_choose_variant.argtypes = [_i, _i, _i, _i, ctypes.POINTER(Variant)]
         L.sfm_get_device_error.argtypes = [_vp, _i, ctypes.POINTER(_i)]
         L.sfm_selective_scan_fold_bwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanGrads), _vp]
+        L.sfm_mixer_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ctypes.c_size_t)]
+        L.sfm_mixer_bwd.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(MixerGrads), _vp, ctypes.c_size_t, _vp]
         for name in ENTRY_POINTS:
             if name not in ("sfm_status_string", "sfm_abi_version", "sfm_last_cuda_error"):
                 getattr(L, name).restype = _i

@@ -212,6 +212,34 @@ BwdParams make_bwd_params(const sfm_scan_args* a, const sfm_scan_grads* g) {
   return p;
 }
 
+sfm_status validate_mixer_grads(const sfm_scan_args* a, const sfm_mixer_grads* g) {
+  if (!g || g->size != sizeof(sfm_mixer_grads)) return SFM_ERR_INVALID_ARG;
+  if (!g->dout || !g->dx || !g->ddt || !g->dA || !g->dB || !g->dC) return SFM_ERR_INVALID_ARG;
+  if ((a->conv_w && !g->dconv_w) || (a->conv_b && a->conv_w && !g->dconv_b) || (a->z && !g->dz) ||
+      (a->Dskip && !g->dDskip) || (a->dt_bias && !g->ddt_bias))
+    return SFM_ERR_INVALID_ARG;
+  if (!aligned16(g->dout)) return SFM_ERR_MISALIGNED;
+  const float* outs[] = {g->dx, g->dconv_w, g->dconv_b, g->ddt, g->dz, g->dA, g->dDskip, g->ddt_bias, g->dB, g->dC};
+  for (const float* o : outs)
+    if (o && (reinterpret_cast<uintptr_t>(o) & 3u)) return SFM_ERR_MISALIGNED;
+  const long long si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);
+  const long long bdl = (long long)a->B * a->D * a->L, bnl = (long long)a->B * a->N * a->L;
+  const long long bdx = (long long)a->B * a->D * (a->aux_init ? a->L - 2 : a->L);
+  const int K = a->conv_w ? a->K : 0;
+  const void* ins[] = {a->x, a->dt, a->z, a->Bm, a->Cm, g->dout, a->A, a->Dskip, a->dt_bias, a->conv_w, a->conv_b};
+  const long long insz[] = {bdx * si, bdl * si, bdl * si, bnl * si, bnl * si, bdl * so, (long long)a->D * a->N * 4,
+                            (long long)a->D * 4, (long long)a->D * 4, (long long)a->D * K * 4, (long long)a->D * 4};
+  const long long outsz[] = {bdx * 4, (long long)a->D * K * 4, (long long)a->D * 4, bdl * 4, bdl * 4,
+                             (long long)a->D * a->N * 4, (long long)a->D * 4, (long long)a->D * 4, bnl * 4, bnl * 4};
+  for (int i = 0; i < 10; ++i) {
+    for (int j = 0; j < 11; ++j)
+      if (overlaps(outs[i], outsz[i], ins[j], insz[j])) return SFM_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 10; ++j)
+      if (overlaps(outs[i], outsz[i], outs[j], outsz[j])) return SFM_ERR_INVALID_ARG;
+  }
+  return SFM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -388,6 +416,52 @@ sfm_status sfm_selective_scan_fold_bwd(const sfm_scan_args* a, const sfm_scan_gr
   BwdParams p = make_bwd_params(a, g);
   bwd_carve(p, static_cast<char*>(ws));
   return cuda_status(launch_bwd(p, a->in_dtype, a->out_dtype, stream));
+}
+
+sfm_status sfm_mixer_bwd_workspace_size(const sfm_scan_args* a, size_t* bytes) {
+  if (!bytes) return SFM_ERR_INVALID_ARG;
+  const sfm_status st = validate_scan(a, true);
+  if (st != SFM_OK) return st;
+  *bytes = mixer_bwd_workspace_bytes(a->B, a->D, a->L, a->N, a->conv_w ? a->K : 1, kBwdDTile);
+  return SFM_OK;
+}
+
+sfm_status sfm_mixer_bwd(const sfm_scan_args* a, const sfm_mixer_grads* g, void* ws, size_t wsb,
+                         sfm_stream_t stream) {
+  sfm_status st = validate_scan(a, true);
+  if (st != SFM_OK) return st;
+  if ((st = validate_mixer_grads(a, g)) != SFM_OK) return st;
+  if (!ws) return SFM_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return SFM_ERR_MISALIGNED;
+  if (wsb < mixer_bwd_workspace_bytes(a->B, a->D, a->L, a->N, a->conv_w ? a->K : 1, kBwdDTile))
+    return SFM_ERR_INVALID_ARG;
+  if (fault_injected()) return SFM_ERR_CUDA;
+  sfm_scan_grads sg;
+  std::memset(&sg, 0, sizeof(sg));
+  sg.dout = g->dout;
+  sg.ddt = g->ddt;
+  sg.dz = g->dz;
+  sg.dA = g->dA;
+  sg.dDskip = g->dDskip;
+  sg.ddt_bias = g->ddt_bias;
+  sg.dB = g->dB;
+  sg.dC = g->dC;
+  BwdParams p = make_bwd_params(a, &sg);
+  p.mixer = 1;
+  p.swap_dout = a->swap_out && a->L >= 2;
+  p.aux = a->aux_init;
+  p.conv = a->conv_w != nullptr;
+  p.K = p.conv ? a->K : 1;
+  p.pad_left = p.conv ? a->pad_left : 0;
+  p.Tx = a->aux_init ? a->L - 2 : a->L;
+  p.x = a->x;
+  p.conv_w = a->conv_w;
+  p.conv_b = p.conv ? a->conv_b : nullptr;
+  p.dx = g->dx;
+  p.dconv_w = g->dconv_w;
+  p.dconv_b = p.conv ? g->dconv_b : nullptr;
+  mixer_bwd_carve(p, static_cast<char*>(ws));
+  return cuda_status(launch_mixer_bwd(p, a->in_dtype, a->out_dtype, stream));
 }
 
 sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* a, const sfm_scan_grads* g,

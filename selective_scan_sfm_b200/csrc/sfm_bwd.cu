@@ -25,7 +25,23 @@ namespace sfm {
 
 __device__ __forceinline__ float sigmoid(float v) { return rcp(1.0f + ex2(-v * kLog2e)); }
 
-template <typename TI, typename TD>
+// xa at position s of row `xr` (aux: the mean at 0 and L-1, x shifted by one inside);
+// zero outside the sample.
+template <typename TI>
+__device__ __forceinline__ float xa_row(const TI* xr, int s, int L, bool aux, float mean) {
+  if (s < 0 || s >= L) return 0.0f;
+  if (aux) return (s == 0 || s == L - 1) ? mean : to_f(xr[s - 1]);
+  return to_f(xr[s]);
+}
+
+template <typename TI>
+__device__ __forceinline__ float conv_pre(const BwdParams& p, const TI* xr, int t, int d, float mean) {
+  float acc = p.conv_b ? p.conv_b[d] : 0.0f;
+  for (int k = 0; k < p.K; ++k) acc = fmaf(p.conv_w[(size_t)d * p.K + k], xa_row(xr, t + k - p.pad_left, p.L, p.aux, mean), acc);
+  return acc;
+}
+
+template <typename TI, typename TD, bool MIXER>
 __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int tile = blockIdx.x, b = blockIdx.y;
@@ -37,7 +53,8 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
   const bool gate = p.z != nullptr, use_sp = p.softplus;
   const size_t row = ((size_t)b * p.D + d) * L;
 
-  const TI* u = static_cast<const TI*>(p.u) + row;
+  const TI* u = MIXER ? nullptr : static_cast<const TI*>(p.u) + row;
+  const float* uw = MIXER ? p.u_ws + row : nullptr;
   const TI* dt = static_cast<const TI*>(p.dt) + row;
   const TI* z = gate ? static_cast<const TI*>(p.z) + row : nullptr;
   const TD* dout = static_cast<const TD*>(p.dout) + row;
@@ -56,12 +73,29 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
     const float v = to_f(dt[t]) + dtb;
     return use_sp ? softplus(v) : v;
   };
-  auto gy_at = [&](int t) { return gate ? to_f(dout[t]) * silu(to_f(z[t])) : to_f(dout[t]); };
+  // the layer output was swapped head<->tail: read its gradient through the same map
+  auto dout_at = [&](int t) {
+    const int i = (MIXER && p.swap_dout) ? (t == 0 ? L - 1 : (t == L - 1 ? 0 : t)) : t;
+    return to_f(dout[i]);
+  };
+  auto gy_at = [&](int t) { return gate ? dout_at(t) * silu(to_f(z[t])) : dout_at(t); };
+  auto u_at = [&](int t) { return MIXER ? uw[t] : to_f(u[t]); };
+
+  if (MIXER && active) {  // the scan input of the layer, once: u = SiLU(conv(xa)) (or xa without conv)
+    const TI* xr = static_cast<const TI*>(p.x) + ((size_t)b * p.D + d) * p.Tx;
+    float mean = 0.0f;
+    if (p.aux) {
+      for (int t = 0; t < p.Tx; ++t) mean += to_f(xr[t]);
+      mean /= (float)p.Tx;
+    }
+    float* uo = p.u_ws + row;
+    for (int t = 0; t < L; ++t) uo[t] = p.conv ? silu(conv_pre(p, xr, t, d, mean)) : xa_row(xr, t, L, p.aux, mean);
+  }
 
   float sum_dsk = 0.0f;
   if (active) {
     for (int t = 0; t < L; ++t) {
-      const float gy = gy_at(t), ut = to_f(u[t]);
+      const float gy = gy_at(t), ut = u_at(t);
       du[t] = gy * dsk;
       ddt[t] = 0.0f;
       if (gate) dz[t] = dsk * ut;
@@ -78,7 +112,7 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
       float h = 0.0f;
       for (int t = 0; t < L; ++t) {
         const float delta = delta_at(t);
-        const float bu = delta * to_f(Bn[t]) * to_f(u[t]);
+        const float bu = delta * to_f(Bn[t]) * u_at(t);
         h = t == 0 ? bu : fmaf(ex2(delta * an * kLog2e), h, bu);
         hb[t] = h;
         if (gate) dz[t] = fmaf(to_f(Cn[t]), h, dz[t]);
@@ -86,7 +120,7 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
       // reverse sweep
       float g = 0.0f, a_next = 0.0f, dA = 0.0f;
       for (int t = L - 1; t >= 0; --t) {
-        const float delta = delta_at(t), gy = gy_at(t), ut = to_f(u[t]), Bv = to_f(Bn[t]);
+        const float delta = delta_at(t), gy = gy_at(t), ut = u_at(t), Bv = to_f(Bn[t]);
         g = fmaf(gy, to_f(Cn[t]), t + 1 < L ? a_next * g : 0.0f);
         cC[t] = gy * hb[t];
         cB[t] = g * delta * ut;
@@ -129,7 +163,7 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
       sum_bias += ds;
       if (gate) {
         const float zt = to_f(z[t]), sg = sigmoid(zt);
-        dz[t] = to_f(dout[t]) * dz[t] * (sg * (1.0f + zt * (1.0f - sg)));
+        dz[t] = dout_at(t) * dz[t] * (sg * (1.0f + zt * (1.0f - sg)));
       }
     }
     p.partD[(size_t)b * p.D + d] = sum_dsk;
@@ -231,7 +265,7 @@ cudaError_t noalloc_scratch(void** out) {
 template <typename TI, typename TD>
 static cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
   const int threads = (p.d_tile + 31) & ~31;
-  bwd_main_kernel<TI, TD><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
+  bwd_main_kernel<TI, TD, false><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t nbc = (size_t)p.B * p.N * p.L;
@@ -246,6 +280,130 @@ cudaError_t launch_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dt
   if (in_dtype == SFM_F32 && dout_dtype == SFM_F32) return launch_bwd_t<float, float>(p, s);
   if (in_dtype == SFM_BF16 && dout_dtype == SFM_BF16) return launch_bwd_t<__nv_bfloat16, __nv_bfloat16>(p, s);
   if (in_dtype == SFM_BF16 && dout_dtype == SFM_F32) return launch_bwd_t<__nv_bfloat16, float>(p, s);
+  return cudaErrorInvalidValue;
+}
+
+// Conv + SiLU (+ aux init) backward, one warp per (b, d) row: dpre = du * SiLU'(pre) (pre
+// recomputed from x), dxa = transposed conv of dpre inside the sample, dx = dxa shifted by
+// the aux token plus the mean's share (dxa[0] + dxa[L-1]) / T; per-row partials of dw, db.
+template <typename TI>
+__global__ void conv_bwd_kernel(const BwdParams p) {
+  const int lane = threadIdx.x & 31;
+  const long long r = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= (long long)p.B * p.D) return;
+  const int d = (int)(r % p.D), L = p.L, Tx = p.Tx, K = p.conv ? p.K : 1, pl = p.conv ? p.pad_left : 0;
+  const TI* xr = static_cast<const TI*>(p.x) + r * Tx;
+  float mean = 0.0f;
+  if (p.aux) {
+    for (int t = lane; t < Tx; t += 32) mean += to_f(xr[t]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mean += __shfl_xor_sync(0xffffffffu, mean, o);
+    mean /= (float)Tx;
+  }
+  float* dp = p.u_ws + r * L;      // u is no longer needed: the row holds dpre
+  const float* du = p.du + r * L;
+  float dw[SFM_MAX_K] = {0.f, 0.f, 0.f, 0.f}, db = 0.0f;
+  for (int t = lane; t < L; t += 32) {
+    float g = du[t];
+    if (p.conv) {
+      const float pre = conv_pre(p, xr, t, d, mean), sg = rcp(1.0f + ex2(-pre * kLog2e));
+      g *= sg * (1.0f + pre * (1.0f - sg));
+#pragma unroll
+      for (int k = 0; k < SFM_MAX_K; ++k)
+        if (k < K) dw[k] = fmaf(g, xa_row(xr, t + k - pl, L, p.aux, mean), dw[k]);
+      db += g;
+    }
+    dp[t] = g;
+  }
+  __syncwarp();
+  auto dxa = [&](int s) {
+    if (!p.conv) return dp[s];
+    float acc = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      const int t = s - k + pl;
+      if (t >= 0 && t < L) acc = fmaf(p.conv_w[(size_t)d * K + k], dp[t], acc);
+    }
+    return acc;
+  };
+  float* dx = p.dx + r * Tx;
+  const float share = p.aux ? (dxa(0) + dxa(L - 1)) / (float)Tx : 0.0f;
+  for (int t = lane; t < Tx; t += 32) dx[t] = dxa(p.aux ? t + 1 : t) + share;
+  if (p.conv) {
+#pragma unroll
+    for (int k = 0; k < SFM_MAX_K; ++k)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dw[k] += __shfl_xor_sync(0xffffffffu, dw[k], o);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) db += __shfl_xor_sync(0xffffffffu, db, o);
+    if (lane == 0) {
+      for (int k = 0; k < K; ++k) p.dw_part[r * K + k] = dw[k];
+      p.db_part[r] = db;
+    }
+  }
+}
+
+// dconv_w[d,k], dconv_b[d]: sum of the per-sample partials in sample order.
+__global__ void conv_reduce_kernel(const BwdParams p) {
+  const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t DK = (size_t)p.D * p.K;
+  if (i < DK) {
+    float s = 0.0f;
+    for (int b = 0; b < p.B; ++b) s += p.dw_part[(size_t)b * DK + i];
+    p.dconv_w[i] = s;
+  }
+  if (i < (size_t)p.D && p.dconv_b) {
+    float s = 0.0f;
+    for (int b = 0; b < p.B; ++b) s += p.db_part[(size_t)b * p.D + i];
+    p.dconv_b[i] = s;
+  }
+}
+
+size_t mixer_bwd_workspace_bytes(int B, int D, int L, int N, int K, int d_tile) {
+  const size_t bdl = (size_t)B * D * L;
+  return bwd_workspace_bytes(B, D, L, N, d_tile) + 2 * align256(bdl * 4) + align256((size_t)B * D * K * 4) +
+         align256((size_t)B * D * 4);
+}
+
+void mixer_bwd_carve(BwdParams& p, char* ws) {
+  bwd_carve(p, ws);
+  size_t o = bwd_workspace_bytes(p.B, p.D, p.L, p.N, p.d_tile);
+  const size_t bdl = (size_t)p.B * p.D * p.L;
+  p.u_ws = reinterpret_cast<float*>(ws + o);
+  o += align256(bdl * 4);
+  p.du = reinterpret_cast<float*>(ws + o);  // the scan input's gradient stays internal
+  o += align256(bdl * 4);
+  p.dw_part = reinterpret_cast<float*>(ws + o);
+  o += align256((size_t)p.B * p.D * (p.K > 0 ? p.K : 1) * 4);
+  p.db_part = reinterpret_cast<float*>(ws + o);
+}
+
+template <typename TI, typename TD>
+static cudaError_t launch_mixer_bwd_t(const BwdParams& p, cudaStream_t s) {
+  const int threads = (p.d_tile + 31) & ~31;
+  bwd_main_kernel<TI, TD, true><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t nbc = (size_t)p.B * p.N * p.L;
+  bwd_reduce_bc_kernel<<<(unsigned)((nbc + 255) / 256), 256, 0, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const size_t np = (size_t)p.D * p.N > (size_t)p.D ? (size_t)p.D * p.N : (size_t)p.D;
+  bwd_reduce_param_kernel<<<(unsigned)((np + 255) / 256), 256, 0, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const long long rows = (long long)p.B * p.D;
+  conv_bwd_kernel<TI><<<(unsigned)((rows + 7) / 8), 256, 0, s>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (p.conv) {
+    const size_t nc = (size_t)p.D * p.K > (size_t)p.D ? (size_t)p.D * p.K : (size_t)p.D;
+    conv_reduce_kernel<<<(unsigned)((nc + 255) / 256), 256, 0, s>>>(p);
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+cudaError_t launch_mixer_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dtype, cudaStream_t s) {
+  if (in_dtype == SFM_F32 && dout_dtype == SFM_F32) return launch_mixer_bwd_t<float, float>(p, s);
+  if (in_dtype == SFM_BF16 && dout_dtype == SFM_BF16) return launch_mixer_bwd_t<__nv_bfloat16, __nv_bfloat16>(p, s);
+  if (in_dtype == SFM_BF16 && dout_dtype == SFM_F32) return launch_mixer_bwd_t<__nv_bfloat16, float>(p, s);
   return cudaErrorInvalidValue;
 }
 

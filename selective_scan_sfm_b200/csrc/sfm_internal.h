@@ -64,6 +64,12 @@ struct BwdParams {
   float *hbuf, *cB, *cC, *partBC, *partA, *partD, *partBias;
   int B, D, L, N, d_tile, ntiles;
   int softplus;
+  // mixer mode (the whole layer): the scan input u = SiLU(conv(xa)) is built from x into
+  // u_ws; the output gradient is read through the head<->tail swap when swap_dout
+  int mixer, swap_dout, aux, conv, K, pad_left, Tx;
+  const void* x;
+  const float *conv_w, *conv_b;
+  float *u_ws, *dx, *dconv_w, *dconv_b, *dw_part, *db_part;
 };
 
 // Launchers (defined in the .cu files).  They only enqueue work; they return the
@@ -81,6 +87,9 @@ cudaError_t read_device_error(cudaStream_t s, int clear, unsigned* value);
 cudaError_t launch_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dtype, cudaStream_t s);
 size_t bwd_workspace_bytes(int B, int D, int L, int N, int d_tile);
 void bwd_carve(BwdParams& p, char* ws);
+size_t mixer_bwd_workspace_bytes(int B, int D, int L, int N, int K, int d_tile);
+void mixer_bwd_carve(BwdParams& p, char* ws);
+cudaError_t launch_mixer_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dtype, cudaStream_t s);
 cudaError_t noalloc_scratch(void** out);  // device address of the built-in workspace
 
 cudaError_t launch_aux_init(const void* x, void* xa, int B, int D, int T, int esize, cudaStream_t s);

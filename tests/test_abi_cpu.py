@@ -25,7 +25,7 @@ def header_entry_points():
 
 def test_exports_every_declared_symbol(L):
     declared = header_entry_points()
-    assert len(declared) >= 12
+    assert len(declared) >= 15
     assert sorted(_abi.ENTRY_POINTS) == declared
     for name in declared:
         assert hasattr(L, name), name
@@ -182,3 +182,21 @@ def test_backward_workspace_query_and_validation(L, inject):
     assert call(bwd_args(), good_grads(du=FAKE + (1 << 24))) == _abi.SFM_ERR_INVALID_ARG  # du aliases dt
     assert call(bwd_args(), good_grads(size=4)) == _abi.SFM_ERR_INVALID_ARG
     assert call(bwd_args(), good_grads(dA=FAKE + (20 << 24) + 2)) == _abi.SFM_ERR_MISALIGNED
+
+
+def test_mixer_backward_validation(L, inject):
+    need = ctypes.c_size_t(0)
+    assert L.sfm_mixer_bwd_workspace_size(ctypes.byref(good_args(swap_out=1)), ctypes.byref(need)) == _abi.SFM_OK
+    g = _abi.MixerGrads()
+    g.size = ctypes.sizeof(_abi.MixerGrads)
+    base = FAKE + (16 << 24)
+    for i, k in enumerate(("dout", "dx", "dconv_w", "dconv_b", "ddt", "dz", "dA", "dDskip", "ddt_bias", "dB", "dC")):
+        setattr(g, k, base + (i << 24))
+    ws = FAKE + (40 << 24)
+    call = lambda a, gg, n=need.value: L.sfm_mixer_bwd(ctypes.byref(a), ctypes.byref(gg), ws, n, None)
+    assert call(good_args(swap_out=1), g) == _abi.SFM_ERR_CUDA       # valid: reaches the launch path
+    assert call(good_args(), g, need.value - 1) == _abi.SFM_ERR_INVALID_ARG
+    g.dconv_w = None
+    assert call(good_args(), g) == _abi.SFM_ERR_INVALID_ARG          # conv given, no dconv_w
+    g.dconv_w = FAKE + (1 << 24)                                      # aliases dt
+    assert call(good_args(), g) == _abi.SFM_ERR_INVALID_ARG

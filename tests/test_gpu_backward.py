@@ -98,3 +98,67 @@ def test_backward_chain_stage3_shape_bf16():
     errs = check_grads(g, ref, TOL["bf16"], TOL["bf16"])
     # fp32 arithmetic on exact bf16 inputs: far inside the bf16 bound
     assert max(errs.values()) < 1e-3, errs
+
+
+# ------------------------------------------------------------------ the whole mixer layer
+
+from selective_scan_sfm_b200 import sfm_mixer_bwd  # noqa: E402
+
+MIXER_ELEM = ("dx", "ddt", "dz", "dB", "dC")
+MIXER_RED = ("dconv_w", "dconv_b", "dA", "dDskip", "ddt_bias")
+
+
+def run_mixer_both(d, dout, aux, swap, pad_left=1, bias=True):
+    dc = to_cuda(d)
+    kw = dict(z=dc["z"], Dskip=dc["Dskip"], dt_bias=dc["dt_bias"], conv_w=dc["conv_w"],
+              conv_b=dc["conv_b"] if bias else None, pad_left=pad_left, aux_init=aux, swap_out=swap)
+    g = sfm_mixer_bwd(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], dout.cuda(), **kw)
+    torch.cuda.synchronize()
+    f = lambda t: t.double().numpy()
+    ref = oracle.mixer_layer_bwd(f(d["x"]), f(d["dt"]), f(d["z"]), f(d["Bm"]), f(d["Cm"]), f(d["A"]),
+                                 f(d["Dskip"]), f(d["dt_bias"]), f(d["conv_w"]),
+                                 f(d["conv_b"]) if bias else None, f(dout), aux_init_in=aux, swap_out=swap,
+                                 pad_left=pad_left)
+    return {k: v.double().cpu().numpy() for k, v in g.items()}, ref
+
+
+def check_mixer(g, ref, tol):
+    errs = {}
+    for k in ref:
+        errs[k] = rel_err(g[k], ref[k]) if k in MIXER_ELEM else normwise(g[k], ref[k])
+    assert set(g) == set(ref), (sorted(g), sorted(ref))
+    bad = {k: e for k, e in errs.items() if e > tol}
+    assert not bad, "mixer gradient errors above bound: %s (all: %s)" % (bad, errs)
+    return errs
+
+
+@pytest.mark.parametrize("aux,swap,pad_left,bias", [(True, True, 1, True), (False, False, 3, True),
+                                                    (True, False, 0, False), (False, True, 2, True)])
+def test_mixer_backward_small_fp32(aux, swap, pad_left, bias):
+    B, D, T, N = 3, 70, 33, 8
+    d = synth.make_inputs(B=B, D=D, T=T, N=N, dtype="f32", seed=4100 + pad_left, aux=aux, random_A=True)
+    L = T + 2 if aux else T
+    dout = synth.make_dout(B, D, L, seed=4100, dtype="f32")
+    g, ref = run_mixer_both(d, dout, aux, swap, pad_left, bias)
+    check_mixer(g, ref, TOL["f32"])
+
+
+def test_mixer_backward_chain_stage3_bf16():
+    """The stage-entry layer of the four-layer chain (aux init, swapped output) at full size."""
+    w = synth.WORKLOADS["chain4_stage3"]
+    d = synth.make_inputs(**w, seed=0)
+    dout = synth.make_dout(w["B"], w["D"], w["T"] + 2, seed=9)
+    g, ref = run_mixer_both(d, dout, True, True)
+    errs = check_mixer(g, ref, TOL["bf16"])
+    assert max(errs.values()) < 1e-3, errs
+
+
+def test_mixer_backward_is_bitwise_reproducible():
+    d = to_cuda(synth.make_inputs(B=4, D=96, T=49, N=16, dtype="bf16", seed=4200))
+    dout = synth.make_dout(4, 96, 51, seed=4200).cuda()
+    run = lambda: sfm_mixer_bwd(d["x"], d["dt"], d["Bm"], d["Cm"], d["A"], dout, z=d["z"], Dskip=d["Dskip"],
+                                dt_bias=d["dt_bias"], conv_w=d["conv_w"], conv_b=d["conv_b"], aux_init=True,
+                                swap_out=True)
+    a, b = run(), run()
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
