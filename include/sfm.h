@@ -166,7 +166,9 @@ typedef struct {
  * independent), so B1 only changes the schedule.
  * Requirements: x, dt, z, Bm, Cm, y 16-byte aligned; 1 <= N <= SFM_MAX_N;
  * 1 <= K <= SFM_MAX_K; 3 <= L <= SFM_MAX_L when aux_init (else 1 <= L); y must not
- * alias an input.  Sources: see the header comment.
+ * alias an input.  One thread per channel (lanes = 1) holds at most 16 states; above
+ * that the lanes mode is chosen (an explicit lanes = 1 is SFM_ERR_UNSUPPORTED).
+ * Sources: see the header comment.
  */
 SFM_API sfm_status sfm_selective_scan_fold(const sfm_scan_args* args, sfm_stream_t stream);
 

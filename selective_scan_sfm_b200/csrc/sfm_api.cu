@@ -114,7 +114,6 @@ sfm_status validate_scan(const sfm_scan_args* a, bool bwd) {
   if (!bwd && !a->y) return SFM_ERR_INVALID_ARG;
   if (a->B < 1 || a->D < 1 || a->L < 1 || a->N < 1) return SFM_ERR_INVALID_ARG;
   if (a->N > SFM_MAX_N || a->L > SFM_MAX_L) return SFM_ERR_UNSUPPORTED;
-  if (a->N > kMaxNFused) return SFM_ERR_UNSUPPORTED;
   if ((a->dt_softplus | a->aux_init | a->swap_out) & ~1) return SFM_ERR_INVALID_ARG;
   if (a->aux_init && a->L < 3) return SFM_ERR_INVALID_ARG;
   if (a->conv_w && (a->K < 1 || a->K > SFM_MAX_K || a->pad_left < 0 || a->pad_left >= a->K))
@@ -346,6 +345,7 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
   const int si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);
   int NP = 2;
   while (NP < a->N) NP <<= 1;
+  p.np = NP;
   if (a->B / p.B2 > kMaxB1) return SFM_ERR_UNSUPPORTED;
   // whole-sample mode: the chunk covers the sample and every slab of every tensor starts
   // on a 16-byte boundary with a size that is a multiple of 16 bytes (bulk-copy rules)
@@ -359,6 +359,14 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
   p.mode = kModeChunk;
   // an explicit channel tile or chunk without explicit lanes asks for one thread per channel
   p.lanes = a->lanes ? a->lanes : ((a->d_tile || a->chunk) ? 1 : v.lanes);
+  // more than kMaxNFused states only fit the lanes mode, which walks the states in pairs
+  if (a->N > kMaxNFused) {
+    if (a->lanes == 1) return SFM_ERR_UNSUPPORTED;
+    if (p.lanes < 2) {
+      p.lanes = 8;
+      if (!a->d_tile) p.d_tile = 16;
+    }
+  }
   if (p.lanes > 1) {
     p.mode = kModeLanes;
     if (!a->d_tile) {

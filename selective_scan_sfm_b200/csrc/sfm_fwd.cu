@@ -769,11 +769,14 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
 // A = 0 on the sample's first token.  The carry between chunks lives in shared memory.
 constexpr int kLaneJ = kLaneTokens;  // tokens per lane per chunk
 
-template <typename TI, typename TO, int NH>
+// The number of state pairs is a runtime value here (states are walked pair by pair in a
+// loop), so one instance serves every N up to SFM_MAX_N.
+template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
   constexpr bool kInPlace = std::is_same<TI, TO>::value;
   constexpr bool kFast = std::is_same<TO, __nv_bfloat16>::value;
-  constexpr int si = sizeof(TI), so = sizeof(TO), NP = 2 * NH, J = kLaneJ;
+  constexpr int si = sizeof(TI), so = sizeof(TO), J = kLaneJ;
+  const int NP = p.np, NH = NP / 2;
   extern __shared__ __align__(16) char smem[];
 
   const int tid = threadIdx.x, nthr = blockDim.x;
@@ -1054,13 +1057,13 @@ static cudaError_t set_smem(Kern k, int bytes, int& have) {
   return e;
 }
 
-template <typename TI, typename TO, int NH>
+template <typename TI, typename TO>
 static cudaError_t launch_lanes(const FwdParams& p, cudaStream_t s) {
   static int have = 48 * 1024;
-  cudaError_t e = set_smem(fwd_lanes_kernel<TI, TO, NH>, p.smem_bytes, have);
+  cudaError_t e = set_smem(fwd_lanes_kernel<TI, TO>, p.smem_bytes, have);
   if (e != cudaSuccess) return e;
   dim3 grid((p.D + p.d_tile - 1) / p.d_tile, p.B / p.B2);
-  fwd_lanes_kernel<TI, TO, NH><<<grid, p.d_tile * p.lanes, p.smem_bytes, s>>>(p);
+  fwd_lanes_kernel<TI, TO><<<grid, p.d_tile * p.lanes, p.smem_bytes, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -1093,7 +1096,6 @@ static cudaError_t launch_t(const FwdParams& p, cudaStream_t s) {
 // N = 16, a choice of how many state pairs take exp2 on the FMA pipe.
 template <typename TI, typename TO, int NH>
 static cudaError_t launch_std(const FwdParams& p, cudaStream_t s) {
-  if (p.mode == kModeLanes) return launch_lanes<TI, TO, NH>(p, s);
   const bool std_path = (p.flags & kConv) && (p.flags & kGate) && (p.flags & kSoftplus) && p.K == 4;
   if (!std_path) return launch_t<TI, TO, NH, false, 0>(p, s);
   if constexpr (NH == 8) {
@@ -1109,6 +1111,7 @@ static cudaError_t launch_std(const FwdParams& p, cudaStream_t s) {
 
 template <typename TI, typename TO>
 static cudaError_t launch_np(const FwdParams& p, int NP, cudaStream_t s) {
+  if (p.mode == kModeLanes) return launch_lanes<TI, TO>(p, s);
   switch (NP) {
     case 2: return launch_std<TI, TO, 1>(p, s);
     case 4: return launch_std<TI, TO, 2>(p, s);

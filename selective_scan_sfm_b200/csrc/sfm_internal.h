@@ -38,6 +38,7 @@ struct FwdParams {
   int mode;            // kModeWhole, kModeChunk or kModeLanes
   int lanes;           // lanes per channel in kModeLanes (chunk = lanes * 8)
   int cpt;             // channels per thread in the whole/chunk modes (1 or 2)
+  int np;              // N padded to a power of two (at least 2)
   int exp2_fma_pairs;  // state pairs per token whose exp2 runs on the FMA pipe (N = 16 path)
   // shared-memory carve-up (bytes), computed on the host
   int x_row, io_row, y_row, smem_bytes;

@@ -162,3 +162,13 @@ def test_mixer_backward_is_bitwise_reproducible():
     a, b = run(), run()
     for k in a:
         assert torch.equal(a[k], b[k]), k
+
+
+def test_backward_large_state_size():
+    d = synth.make_inputs(B=2, D=40, T=30, N=32, dtype="f32", seed=4300, aux=False, random_A=True)
+    dout = synth.make_dout(2, 40, 30, seed=4300, dtype="f32")
+    g, ref = run_both(d, dout)
+    check_grads(g, ref, TOL["f32"], TOL["f32"])
+    d2 = synth.make_inputs(B=2, D=40, T=30, N=32, dtype="f32", seed=4301, random_A=True)
+    g2, ref2 = run_mixer_both(d2, synth.make_dout(2, 40, 32, seed=4301, dtype="f32"), True, True)
+    check_mixer(g2, ref2, TOL["f32"])

@@ -294,3 +294,18 @@ def test_two_channels_per_thread(B, D, T, N, dtype, d_tile, chunk):
         assert rel_err(fs.double().cpu().numpy(), ref_state) <= TOL[dtype]
         y1 = fused(dc, swap_out=swap, d_tile=d_tile, chunk=chunk, chans_per_thread=1, B1=B)
         assert rel_err(y.double().cpu().numpy(), y1.double().cpu().numpy()) <= TOL[dtype]
+
+
+# ------------------------------------------------------------------ state sizes above 16 (lanes mode)
+
+@pytest.mark.parametrize("N,dtype", [(24, "f32"), (32, "bf16"), (64, "f32")])
+def test_large_state_sizes(N, dtype):
+    d = synth.make_inputs(B=3, D=40, T=70, N=N, dtype=dtype, seed=9000 + N, random_A=True)
+    dc = to_cuda(d)
+    fs = torch.full((3, 40, N), float("nan"), device="cuda")
+    y = fused(dc, swap_out=True, final_state=fs)  # routed to lanes mode automatically
+    ref, ref_state = oracle_layer(d, swap_out=True, want_state=True)
+    check(y, ref, dtype, "N=%d" % N)
+    assert rel_err(fs.double().cpu().numpy(), ref_state) <= TOL[dtype]
+    with pytest.raises(SfmError, match="UNSUPPORTED"):
+        fused(dc, lanes=1, d_tile=32)  # one thread per channel holds at most 16 states
