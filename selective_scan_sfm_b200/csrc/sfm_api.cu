@@ -363,7 +363,7 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
   if (a->N > kMaxNFused) {
     if (a->lanes == 1) return SFM_ERR_UNSUPPORTED;
     if (p.lanes < 2) {
-      p.lanes = 8;
+      p.lanes = 4;
       if (!a->d_tile) p.d_tile = 16;
     }
   }
@@ -374,11 +374,24 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
       if (p.d_tile * p.lanes < 32) p.d_tile = 32 / p.lanes;
     }
     if (p.d_tile * p.lanes > 256 || (p.d_tile * p.lanes) % 32 != 0) return SFM_ERR_UNSUPPORTED;
-    p.chunk = p.lanes * kLaneTokens;
-    p.x_row = fwd_x_row(p.chunk, 4, si);
-    p.io_row = fwd_io_row(p.chunk, si);
-    p.y_row = fwd_y_row(p.chunk, so);
-    p.smem_bytes = fwd_lanes_smem(p, si, so, NP);
+    auto shape = [&]() {
+      p.chunk = p.lanes * kLaneTokens;
+      p.x_row = fwd_x_row(p.chunk, 4, si);
+      p.io_row = fwd_io_row(p.chunk, si);
+      p.y_row = fwd_y_row(p.chunk, so);
+      p.smem_bytes = fwd_lanes_smem(p, si, so, NP);
+    };
+    shape();
+    // automatic shapes shrink (fewer lanes, then fewer channels) until the smem fits
+    while (p.smem_bytes > fwd_max_smem() && !a->lanes && p.lanes > 2) {
+      p.lanes /= 2;
+      if (!a->d_tile) p.d_tile = (p.d_tile * 2 * p.lanes <= 256) ? p.d_tile * 2 : p.d_tile;
+      shape();
+    }
+    while (p.smem_bytes > fwd_max_smem() && !a->d_tile && p.d_tile * p.lanes > 32) {
+      p.d_tile /= 2;
+      shape();
+    }
     if (p.smem_bytes > fwd_max_smem()) return SFM_ERR_UNSUPPORTED;
   } else if (p.chunk >= a->L && aligned) {
     p.mode = kModeWhole;

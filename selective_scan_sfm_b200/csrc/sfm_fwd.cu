@@ -760,28 +760,32 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
 // ------------------------------------------------------------------ lanes mode (P > 1)
 //
 // For long samples and few channels (B*D too small to fill the GPU with one thread per
-// channel), P lanes share a channel and split each chunk of S = P*J tokens: lane l owns
-// tokens [l*J, (l+1)*J).  Per pair of states, each lane scans its J tokens locally as
-// (A, B) pairs -- A the product of the decays, B the state reached from zero -- then the
-// P lanes combine their aggregates with a warp-shuffle inclusive scan under
-//   (A1, B1) o (A2, B2) = (A1*A2, A2*B1 + B2),
-// and each lane rebuilds its states from the carry that enters it.  A reset is simply
-// A = 0 on the sample's first token.  The carry between chunks lives in shared memory.
+// channel), and for more than 16 states, P lanes share a channel and split each chunk of
+// S = P*J tokens: lane l owns tokens [l*J, (l+1)*J).  Per pair of states each lane
+//   1. runs its J tokens from a zero state, keeping the decays Abar_j and accumulating the
+//      aggregate (A, B): A the product of the decays, B the state reached from zero;
+//   2. combines the aggregates of the P lanes with a warp-shuffle inclusive scan under
+//        (A1, B1) o (A2, B2) = (A1*A2, A2*B1 + B2),
+//      to get the state entering its tokens from the chunk's carry;
+//   3. replays its J tokens from that state with the kept decays (no second exp) and
+//      accumulates C*h into the outputs.
+// A reset is simply A = 0 on the sample's first token.  The carry between chunks lives
+// in shared memory; staging is double-buffered over (sample, chunk) steps like the
+// chunked mode.  The number of state pairs is a run-time value, so one instance serves
+// every N up to SFM_MAX_N.
 constexpr int kLaneJ = kLaneTokens;  // tokens per lane per chunk
 
-// The number of state pairs is a runtime value here (states are walked pair by pair in a
-// loop), so one instance serves every N up to SFM_MAX_N.
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
   constexpr bool kInPlace = std::is_same<TI, TO>::value;
   constexpr bool kFast = std::is_same<TO, __nv_bfloat16>::value;
   constexpr int si = sizeof(TI), so = sizeof(TO), J = kLaneJ;
-  const int NP = p.np, NH = NP / 2;
   extern __shared__ __align__(16) char smem[];
 
+  const int NP = p.np, NH = NP / 2;
   const int tid = threadIdx.x, nthr = blockDim.x;
-  const int P = p.lanes, lane = tid % P, c = tid / P;  // channel within the tile, lane within the channel
-  const int nch = nthr / P;                              // channels per CTA (= d_tile)
+  const int P = p.lanes, lane = tid % P, c = tid / P;
+  const int nch = nthr / P;
   const int d0 = blockIdx.x * p.d_tile;
   const int dcount = min(p.d_tile, p.D - d0);
   const int b1 = blockIdx.y;
@@ -792,16 +796,18 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
   const bool swap = p.flags & kSwapOut;
   const int K = o.conv ? o.K : 1, pl = o.pl;
   const unsigned gmask = (P == 32) ? 0xffffffffu : (((1u << P) - 1u) << ((tid & 31) / P * P));
+  const int lgS = 31 - __clz(S);
 
-  char* xs = smem;
-  char* dts = xs + p.d_tile * p.x_row;
-  char* zs = dts + p.d_tile * p.io_row;
-  char* bs = zs + (o.gate ? p.d_tile * p.io_row : 0);
-  char* cs = bs + N * p.io_row;
-  float* bcn = reinterpret_cast<float*>(cs + N * p.io_row);  // [2*NP][S]: B rows, then C rows
-  float* a_s = bcn + 2 * NP * S;                             // [d_tile][NP]: A * log2(e)
-  float* carry = a_s + p.d_tile * NP;                        // [d_tile][NP]: state entering the chunk
+  const int stage_bytes = p.d_tile * p.x_row + p.d_tile * p.io_row * (o.gate ? 2 : 1) + 2 * N * p.io_row;
+  float* bcn = reinterpret_cast<float*>(smem + 2 * stage_bytes);  // [2*NP][S]: B rows, then C rows
+  float* a_s = bcn + 2 * NP * S;                                   // [d_tile][NP]: A * log2(e)
+  float* carry = a_s + p.d_tile * NP;                              // [d_tile][NP]: state entering the chunk
   char* ys = reinterpret_cast<char*>(carry + p.d_tile * NP);
+  auto xs_of = [&](int st) { return smem + st * stage_bytes; };
+  auto dts_of = [&](int st) { return xs_of(st) + p.d_tile * p.x_row; };
+  auto zs_of = [&](int st) { return dts_of(st) + p.d_tile * p.io_row; };
+  auto bs_of = [&](int st) { return zs_of(st) + (o.gate ? p.d_tile * p.io_row : 0); };
+  auto cs_of = [&](int st) { return bs_of(st) + N * p.io_row; };
 
   for (int e = tid; e < p.d_tile * NP; e += nthr) {
     const int cc = e / NP, n = e % NP;
@@ -824,71 +830,99 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
   const char* cg = static_cast<const char*>(p.Cm);
   TO* yg = static_cast<TO*>(p.y);
   const int nchunks = (L + S - 1) / S;
+  const int nsteps = p.B2 * nchunks;
 
-  for (int j = 0; j < p.B2; ++j) {
-    const int b = b1 * p.B2 + j;
+  auto x_window = [&](int t0, int cnt, int& xlo, int& xhi) {
+    const int slo = t0 - pl - o.off, shi = t0 + cnt - 1 + (K - 1 - pl) - o.off;
+    xlo = max(slo, 0);
+    xhi = min(shi + 1, Tx);
+  };
+  // the lanes of a channel share its rows' granules; channel groups share the B, C rows
+  auto stage = [&](int st, int buf) {
+    const int b = b1 * p.B2 + st / nchunks, t0 = (st % nchunks) * S, cnt = min(S, L - t0);
+    const long long myrow = (long long)b * p.D + d0 + c;
+    int xlo, xhi;
+    x_window(t0, cnt, xlo, xhi);
+    if (active) {
+      copy_span_async(xs_of(buf) + c * p.x_row, xg, myrow * Tx + xlo, xhi - xlo, si, x_bytes, lane, P);
+      copy_span_async(dts_of(buf) + c * p.io_row, dtg, myrow * L + t0, cnt, si, io_bytes, lane, P);
+      if (o.gate) copy_span_async(zs_of(buf) + c * p.io_row, zg, myrow * L + t0, cnt, si, io_bytes, lane, P);
+    }
+    for (int r = c; r < 2 * N; r += nch) {
+      const int n = r % N;
+      const long long e0 = ((long long)b * N + n) * L + t0;
+      copy_span_async((r < N ? bs_of(buf) : cs_of(buf)) + n * p.io_row, r < N ? bg : cg, e0, cnt, si, bc_bytes,
+                      lane, P);
+    }
+    cp_async_commit();
+  };
+
+  float mean = 0.0f, head_val = 0.0f;
+  stage(0, 0);
+  for (int st = 0; st < nsteps; ++st) {
+    const int buf = st & 1;
+    const int jsam = st / nchunks, kc = st % nchunks;
+    const int b = b1 * p.B2 + jsam;
     const long long row0 = (long long)b * p.D + d0;
     const long long myrow = row0 + c;
-    // aux mean: the channel's lanes sum strided parts of its row, then combine
-    float mean = 0.0f;
-    if (o.aux) {
-      float s0 = 0.0f;
-      if (active) {
-        const TI* xr = reinterpret_cast<const TI*>(xg) + myrow * Tx;
-        for (int t = lane; t < Tx; t += P) s0 += to_f(xr[t]);
-      }
-      for (int off = P / 2; off > 0; off >>= 1) s0 += __shfl_xor_sync(gmask, s0, off, P);
-      mean = s0 / (float)Tx;
-    }
-    for (int e = tid; e < p.d_tile * NP; e += nthr) carry[e] = 0.0f;
-    float head_val = 0.0f;  // output of token 0 (held by lane 0), written to L-1 when swapping
-
-    for (int kc = 0; kc < nchunks; ++kc) {
-      const int t0 = kc * S, cnt = min(S, L - t0);
-      const int slo = t0 - pl - o.off, shi = t0 + cnt - 1 + (K - 1 - pl) - o.off;
-      const int xlo = max(slo, 0), xhi = min(shi + 1, Tx);
-      // ---- stage: the lanes of a channel share its rows' granules
-      if (active) {
-        copy_span_async(xs + c * p.x_row, xg, myrow * Tx + xlo, xhi - xlo, si, x_bytes, lane, P);
-        copy_span_async(dts + c * p.io_row, dtg, myrow * L + t0, cnt, si, io_bytes, lane, P);
-        if (o.gate) copy_span_async(zs + c * p.io_row, zg, myrow * L + t0, cnt, si, io_bytes, lane, P);
-      }
-      for (int r = c; r < 2 * N; r += nch) {
-        const int n = r % N;
-        const long long e0 = ((long long)b * N + n) * L + t0;
-        copy_span_async((r < N ? bs : cs) + n * p.io_row, r < N ? bg : cg, e0, cnt, si, bc_bytes, lane, P);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      __syncthreads();
-      // ---- B, C -> fp32 [2*NP][S], zero past the chunk end and for padded states (S = P*J
-      // is a power of two)
-      const int lgS = 31 - __clz(S);
-      for (int e = tid; e < 2 * NP * S; e += nthr) {
-        const int r = e >> lgS, i = e & (S - 1), n = r % NP;
-        float v = 0.0f;
-        if (n < N && i < cnt) {
-          const char* raw = (r < NP ? bs : cs) + n * p.io_row;
-          const int hb = (int)(((unsigned)(((long long)b * N + n) * L + t0) * si) & 15u);
-          v = to_f(*reinterpret_cast<const TI*>(raw + hb + i * si));
+    const int t0 = kc * S, cnt = min(S, L - t0);
+    int xlo, xhi;
+    x_window(t0, cnt, xlo, xhi);
+    if (kc == 0) {  // a new sample: zero carry; the aux mean from the whole x row
+      if (o.aux) {
+        float s0 = 0.0f, s1 = 0.0f;
+        if (active) {
+          const TI* xr = reinterpret_cast<const TI*>(xg) + myrow * Tx;
+          int t = lane;
+          for (; t + P < Tx; t += 2 * P) {
+            s0 += to_f(xr[t]);
+            s1 += to_f(xr[t + P]);
+          }
+          if (t < Tx) s0 += to_f(xr[t]);
         }
-        bcn[e] = v;
+        s0 += s1;
+        for (int off = P / 2; off > 0; off >>= 1) s0 += __shfl_xor_sync(gmask, s0, off, P);
+        mean = s0 / (float)Tx;
       }
-      __syncthreads();
+      for (int e = tid; e < p.d_tile * NP; e += nthr) carry[e] = 0.0f;
+    }
+    if (st + 1 < nsteps) {
+      stage(st + 1, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    // ---- B, C -> fp32 [2*NP][S], zero past the chunk end and for padded states
+    for (int e = tid; e < 2 * NP * S; e += nthr) {
+      const int r = e >> lgS, i = e & (S - 1), n = r & (NP - 1);
+      float v = 0.0f;
+      if (n < N && i < cnt) {
+        const char* raw = (r < NP ? bs_of(buf) : cs_of(buf)) + n * p.io_row;
+        const int hb = (int)(((unsigned)(((long long)b * N + n) * L + t0) * si) & 15u);
+        v = to_f(*reinterpret_cast<const TI*>(raw + hb + i * si));
+      }
+      bcn[e] = v;
+    }
+    __syncthreads();
 
-      if (active) {
-        const TI* xr = reinterpret_cast<const TI*>(xs + c * p.x_row + span_head(myrow * Tx + xlo, si));
-        const int hd = span_head(myrow * L + t0, si);
-        const TI* dtr = reinterpret_cast<const TI*>(dts + c * p.io_row + hd);
-        const TI* zr = o.gate ? reinterpret_cast<const TI*>(zs + c * p.io_row + hd) : dtr;
-        TO* yr = kInPlace ? reinterpret_cast<TO*>(dts + c * p.io_row + hd) : reinterpret_cast<TO*>(ys + c * p.y_row);
-        const int i0 = lane * J;  // chunk-relative first token of this lane
+    if (active) {
+      const TI* xr = reinterpret_cast<const TI*>(xs_of(buf) + c * p.x_row + span_head(myrow * Tx + xlo, si));
+      const int hd = span_head(myrow * L + t0, si);
+      char* dtrow = dts_of(buf) + c * p.io_row;  // the granule row: element 0 at byte hd
+      const TI* dtr = reinterpret_cast<const TI*>(dtrow + hd);
+      const TI* zr = o.gate ? reinterpret_cast<const TI*>(zs_of(buf) + c * p.io_row + hd) : dtr;
+      TO* yr = kInPlace ? reinterpret_cast<TO*>(dtrow + hd) : reinterpret_cast<TO*>(ys + c * p.y_row);
+      const int i0 = lane * J;  // chunk-relative first token of this lane
 
-        // ---- per-token inputs of the lane's J tokens (identity (A,B) = (1,0) past the end)
-        float dl[J], du[J], yv[J], gz[J];
+      // ---- per-token inputs of the lane's J tokens (identity (A,B) = (1,0) past the end)
+      float dl[J], du[J];
+      float2 yacc[J];
+      {
         float xw[J + 3];
 #pragma unroll
-        for (int q = 0; q < J + 3; ++q) xw[q] = (q < J || o.conv) ? xa_at<TI>(o, xr, xlo, xhi, mean, t0 + i0 + q - pl) : 0.0f;
+        for (int q = 0; q < J + 3; ++q)
+          xw[q] = (q < J || o.conv) ? xa_at<TI>(o, xr, xlo, xhi, mean, t0 + i0 + q - pl) : 0.0f;
 #pragma unroll
         for (int jj = 0; jj < J; ++jj) {
           const bool valid = i0 + jj < cnt;
@@ -906,101 +940,116 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
           const float delta = valid ? (o.sp ? (kFast ? softplus_fast(v) : softplus(v)) : v) : 0.0f;
           dl[jj] = delta;
           du[jj] = valid ? delta * u : 0.0f;
-          yv[jj] = dsk * u;
-          gz[jj] = (o.gate && valid) ? (kFast ? silu_fast(to_f(zr[i0 + jj])) : silu(to_f(zr[i0 + jj]))) : 1.0f;
+          yacc[jj] = make_float2(dsk * u, 0.0f);
         }
-        const bool reset0 = (t0 + i0 == 0);  // the sample's first token lives in lane 0 of chunk 0
+      }
+      const bool reset0 = (t0 + i0 == 0);  // the sample's first token lives in lane 0 of chunk 0
 
-        float2 yacc[J];
-#pragma unroll
-        for (int jj = 0; jj < J; ++jj) yacc[jj] = make_float2(0.f, 0.f);
 #pragma unroll 1
-        for (int k = 0; k < NH; ++k) {
-          const float2 A2 = make_float2(a_s[c * NP + 2 * k], a_s[c * NP + 2 * k + 1]);
-          const float* B0 = bcn + (2 * k) * S + i0;
-          const float* B1r = bcn + (2 * k + 1) * S + i0;
-          const float* C0 = bcn + (NP + 2 * k) * S + i0;
-          const float* C1r = bcn + (NP + 2 * k + 1) * S + i0;
-          float2 Ac[J], Bc[J];
+      for (int k = 0; k < NH; ++k) {
+        const float2 A2 = *reinterpret_cast<const float2*>(a_s + c * NP + 2 * k);
+        float Bv0[J], Bv1[J];
 #pragma unroll
-          for (int jj = 0; jj < J; ++jj) {
-            float2 a = __fmul2_rn(make_float2(dl[jj], dl[jj]), A2);
-            a.x = ex2(a.x);
-            a.y = ex2(a.y);
-            if (jj == 0 && reset0) a = make_float2(0.f, 0.f);
-            const float2 bb = __fmul2_rn(make_float2(B0[jj], B1r[jj]), make_float2(du[jj], du[jj]));
-            if (jj == 0) {
-              Ac[0] = a;
-              Bc[0] = bb;
-            } else {
-              Bc[jj] = __ffma2_rn(a, Bc[jj - 1], bb);
-              Ac[jj] = __fmul2_rn(a, Ac[jj - 1]);
-            }
-          }
-          // inclusive scan of the lanes' aggregates, within the channel's P lanes
-          float2 Ai = Ac[J - 1], Bi = Bc[J - 1];
-          for (int off = 1; off < P; off <<= 1) {
-            const float2 Ap = make_float2(__shfl_up_sync(gmask, Ai.x, off, P), __shfl_up_sync(gmask, Ai.y, off, P));
-            const float2 Bp = make_float2(__shfl_up_sync(gmask, Bi.x, off, P), __shfl_up_sync(gmask, Bi.y, off, P));
-            if (lane >= off) {
-              Bi = __ffma2_rn(Ai, Bp, Bi);
-              Ai = __fmul2_rn(Ai, Ap);
-            }
-          }
-          // exclusive prefix -> the state entering this lane's tokens
-          float2 Ae = make_float2(__shfl_up_sync(gmask, Ai.x, 1, P), __shfl_up_sync(gmask, Ai.y, 1, P));
-          float2 Be = make_float2(__shfl_up_sync(gmask, Bi.x, 1, P), __shfl_up_sync(gmask, Bi.y, 1, P));
-          if (lane == 0) {
-            Ae = make_float2(1.f, 1.f);
-            Be = make_float2(0.f, 0.f);
-          }
-          const float2 hc = make_float2(carry[c * NP + 2 * k], carry[c * NP + 2 * k + 1]);
-          const float2 hin = __ffma2_rn(Ae, hc, Be);
-          __syncwarp(gmask);
-          if (lane == P - 1) {  // state leaving the chunk = carry of the next one
-            const float2 hout = __ffma2_rn(Ai, hc, Bi);
-            carry[c * NP + 2 * k] = hout.x;
-            carry[c * NP + 2 * k + 1] = hout.y;
-          }
+        for (int q = 0; q < J; q += 4) {
+          const float4 u0 = *reinterpret_cast<const float4*>(bcn + (2 * k) * S + i0 + q);
+          const float4 u1 = *reinterpret_cast<const float4*>(bcn + (2 * k + 1) * S + i0 + q);
+          Bv0[q] = u0.x; Bv0[q + 1] = u0.y; Bv0[q + 2] = u0.z; Bv0[q + 3] = u0.w;
+          Bv1[q] = u1.x; Bv1[q + 1] = u1.y; Bv1[q + 2] = u1.z; Bv1[q + 3] = u1.w;
+        }
+        // 1. the lane's decays and its aggregate from a zero state
+        float2 a[J];
+        float2 Ar = make_float2(1.f, 1.f), Br = make_float2(0.f, 0.f);
 #pragma unroll
-          for (int jj = 0; jj < J; ++jj) {
-            const float2 h = __ffma2_rn(Ac[jj], hin, Bc[jj]);
-            yacc[jj] = __ffma2_rn(make_float2(C0[jj], C1r[jj]), h, yacc[jj]);
+        for (int jj = 0; jj < J; ++jj) {
+          float2 aj = __fmul2_rn(make_float2(dl[jj], dl[jj]), A2);
+          aj.x = ex2(aj.x);
+          aj.y = ex2(aj.y);
+          if (jj == 0 && reset0) aj = make_float2(0.f, 0.f);
+          a[jj] = aj;
+          const float2 bj = __fmul2_rn(make_float2(Bv0[jj], Bv1[jj]), make_float2(du[jj], du[jj]));
+          Br = __ffma2_rn(aj, Br, bj);
+          Ar = __fmul2_rn(aj, Ar);
+        }
+        // 2. inclusive scan of the lanes' aggregates within the channel's P lanes
+        float2 Ai = Ar, Bi = Br;
+        for (int off = 1; off < P; off <<= 1) {
+          const float2 Ap = make_float2(__shfl_up_sync(gmask, Ai.x, off, P), __shfl_up_sync(gmask, Ai.y, off, P));
+          const float2 Bp = make_float2(__shfl_up_sync(gmask, Bi.x, off, P), __shfl_up_sync(gmask, Bi.y, off, P));
+          if (lane >= off) {
+            Bi = __ffma2_rn(Ai, Bp, Bi);
+            Ai = __fmul2_rn(Ai, Ap);
           }
+        }
+        float2 Ae = make_float2(__shfl_up_sync(gmask, Ai.x, 1, P), __shfl_up_sync(gmask, Ai.y, 1, P));
+        float2 Be = make_float2(__shfl_up_sync(gmask, Bi.x, 1, P), __shfl_up_sync(gmask, Bi.y, 1, P));
+        if (lane == 0) {
+          Ae = make_float2(1.f, 1.f);
+          Be = make_float2(0.f, 0.f);
+        }
+        const float2 hc = *reinterpret_cast<const float2*>(carry + c * NP + 2 * k);
+        float2 h = __ffma2_rn(Ae, hc, Be);  // the state entering this lane's tokens
+        __syncwarp(gmask);
+        if (lane == P - 1) *reinterpret_cast<float2*>(carry + c * NP + 2 * k) = __ffma2_rn(Ai, hc, Bi);
+        // 3. replay from the entering state with the kept decays
+        float Cv0[J], Cv1[J];
+#pragma unroll
+        for (int q = 0; q < J; q += 4) {
+          const float4 u0 = *reinterpret_cast<const float4*>(bcn + (NP + 2 * k) * S + i0 + q);
+          const float4 u1 = *reinterpret_cast<const float4*>(bcn + (NP + 2 * k + 1) * S + i0 + q);
+          Cv0[q] = u0.x; Cv0[q + 1] = u0.y; Cv0[q + 2] = u0.z; Cv0[q + 3] = u0.w;
+          Cv1[q] = u1.x; Cv1[q + 1] = u1.y; Cv1[q + 2] = u1.z; Cv1[q + 3] = u1.w;
         }
 #pragma unroll
         for (int jj = 0; jj < J; ++jj) {
-          const int i = i0 + jj;
-          if (i >= cnt) continue;
-          const float yo = (yacc[jj].x + yacc[jj].y + yv[jj]) * gz[jj];
-          const int t = t0 + i;
-          if (swap && t == 0) head_val = yo;
-          if (swap && t == L - 1)
-            yg[myrow * L] = from_f<TO>(yo);  // the tail output becomes the next head
-          else
-            yr[i] = from_f<TO>(yo);
-        }
-        if (swap && t0 + cnt == L) {
-          // token 0's output sits in lane 0; the lane that owns token L-1 stores it there
-          const float hv = __shfl_sync(gmask, head_val, 0, P);
-          if (lane == (cnt - 1) / J) yr[cnt - 1] = from_f<TO>(hv);
+          const float2 bj = __fmul2_rn(make_float2(Bv0[jj], Bv1[jj]), make_float2(du[jj], du[jj]));
+          h = __ffma2_rn(a[jj], h, bj);
+          yacc[jj] = __ffma2_rn(make_float2(Cv0[jj], Cv1[jj]), h, yacc[jj]);
         }
       }
-      __syncthreads();
-      // ---- store the chunk's outputs, coalesced along rows
+#pragma unroll
+      for (int jj = 0; jj < J; ++jj) {
+        const int i = i0 + jj;
+        if (i >= cnt) continue;
+        float yo = yacc[jj].x + yacc[jj].y;
+        if (o.gate) {
+          const float zf = to_f(zr[i]);
+          yo *= kFast ? silu_fast(zf) : silu(zf);
+        }
+        const int t = t0 + i;
+        if (swap && t == 0) head_val = yo;
+        if (swap && t == L - 1)
+          yg[myrow * L] = from_f<TO>(yo);  // the tail output becomes the next head
+        else
+          yr[i] = from_f<TO>(yo);
+      }
+      if (swap && t0 + cnt == L) {
+        // token 0's output sits in lane 0; the lane that owns token L-1 stores it there
+        const float hv = __shfl_sync(gmask, head_val, 0, P);
+        if (lane == (cnt - 1) / J) yr[cnt - 1] = from_f<TO>(hv);
+      }
+      __syncwarp(gmask);
+      if (kInPlace && i0 < cnt) {  // each lane writes its own tokens back, 16-byte stores where aligned
+        const int off = hd + i0 * si;
+        store_row<TO>(yg, myrow * L + t0 + i0, dtrow + (off & ~15), min(J, cnt - i0), swap && t0 + i0 == 0);
+      }
+      if (p.final_state && kc == nchunks - 1) {
+        __syncwarp(gmask);
+        if (lane == 0) {
+          float* fs = p.final_state + ((size_t)b * p.D + d) * N;
+          for (int n = 0; n < N; ++n) fs[n] = carry[c * NP + n];
+        }
+      }
+    }
+    __syncthreads();  // this step's buffer and bcn are free for the next steps
+    if (!kInPlace) {
       for (int r = tid / 32; r < dcount; r += nthr / 32) {
-        const long long rr = row0 + r;
-        const char* src = kInPlace ? dts + r * p.io_row + span_head(rr * L + t0, si) : ys + r * p.y_row;
-        TO* dst = yg + rr * L + t0;
+        const char* src = ys + r * p.y_row;
+        TO* dst = yg + (row0 + r) * L + t0;
         for (int i = tid % 32; i < cnt; i += 32)
           if (!(swap && t0 + i == 0)) dst[i] = *reinterpret_cast<const TO*>(src + i * so);
       }
+      __syncthreads();
     }
-    if (p.final_state && active && lane == 0) {
-      float* fs = p.final_state + ((size_t)b * p.D + d) * N;
-      for (int n = 0; n < N; ++n) fs[n] = carry[c * NP + n];
-    }
-    __syncthreads();
   }
 }
 
@@ -1035,6 +1084,7 @@ int fwd_lanes_smem(const FwdParams& p, int si, int so, int NP) {
   s += (long long)p.d_tile * p.x_row;
   s += (long long)p.d_tile * p.io_row * (gate ? 2 : 1);
   s += 2LL * p.N * p.io_row;
+  s *= 2;                          // two staging buffers
   s += 2LL * NP * p.chunk * 4;     // B, C in fp32
   s += 2LL * p.d_tile * NP * 4;    // A * log2(e), carry
   if (si != so) s += (long long)p.d_tile * p.y_row;

@@ -36,7 +36,7 @@ struct FwdParams {
   int chunk;           // tokens staged per step of the walk
   int flags;
   int mode;            // kModeWhole, kModeChunk or kModeLanes
-  int lanes;           // lanes per channel in kModeLanes (chunk = lanes * 8)
+  int lanes;           // lanes per channel in kModeLanes (chunk = lanes * kLaneTokens)
   int cpt;             // channels per thread in the whole/chunk modes (1 or 2)
   int np;              // N padded to a power of two (at least 2)
   int exp2_fma_pairs;  // state pairs per token whose exp2 runs on the FMA pipe (N = 16 path)
@@ -48,7 +48,7 @@ struct FwdParams {
 constexpr int kModeChunk = 0;
 constexpr int kModeWhole = 1;
 constexpr int kModeLanes = 2;  // P lanes per channel split the tokens (warp-shuffle scan)
-constexpr int kLaneTokens = 8; // tokens per lane per chunk in kModeLanes
+constexpr int kLaneTokens = 16; // tokens per lane per chunk in kModeLanes
 
 struct BwdParams {
   const void* u;
