@@ -795,12 +795,17 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
   const Opts o = make_opts(p);
   const bool swap = p.flags & kSwapOut;
   const int K = o.conv ? o.K : 1, pl = o.pl;
-  const unsigned gmask = (P == 32) ? 0xffffffffu : (((1u << P) - 1u) << ((tid & 31) / P * P));
-  const int lgS = 31 - __clz(S);
+  // every thread of a warp runs the lane scan (channels past D compute on staged rows that
+  // are never stored), so the shuffles take the full mask
+  constexpr unsigned gmask = 0xffffffffu;
 
   const int stage_bytes = p.d_tile * p.x_row + p.d_tile * p.io_row * (o.gate ? 2 : 1) + 2 * N * p.io_row;
-  float* bcn = reinterpret_cast<float*>(smem + 2 * stage_bytes);  // [2*NP][S]: B rows, then C rows
-  float* a_s = bcn + 2 * NP * S;                                   // [d_tile][NP]: A * log2(e)
+  // B and C in fp32, pair-interleaved per lane: [2][NH][P][LS] with (state 2k, state 2k+1) adjacent
+  // for each token, so a lane's J tokens of one state pair are 2J consecutive floats; the
+  // 4-float pad per lane segment spreads the lanes of a channel over distinct banks.
+  constexpr int LS = 2 * J + 4;
+  float* bcn = reinterpret_cast<float*>(smem + 2 * stage_bytes);
+  float* a_s = bcn + 2 * NH * P * LS;                              // [d_tile][NP]: A * log2(e)
   float* carry = a_s + p.d_tile * NP;                              // [d_tile][NP]: state entering the chunk
   char* ys = reinterpret_cast<char*>(carry + p.d_tile * NP);
   auto xs_of = [&](int st) { return smem + st * stage_bytes; };
@@ -893,20 +898,23 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
       cp_async_wait<0>();
     }
     __syncthreads();
-    // ---- B, C -> fp32 [2*NP][S], zero past the chunk end and for padded states
-    for (int e = tid; e < 2 * NP * S; e += nthr) {
-      const int r = e >> lgS, i = e & (S - 1), n = r & (NP - 1);
-      float v = 0.0f;
-      if (n < N && i < cnt) {
-        const char* raw = (r < NP ? bs_of(buf) : cs_of(buf)) + n * p.io_row;
-        const int hb = (int)(((unsigned)(((long long)b * N + n) * L + t0) * si) & 15u);
-        v = to_f(*reinterpret_cast<const TI*>(raw + hb + i * si));
+    // ---- B, C -> fp32, one warp per row; zero past the chunk end and for padded states
+    for (int r = tid / 32; r < 2 * NP; r += nthr / 32) {
+      const int side = r >= NP, n = r - side * NP;
+      float* dst = bcn + (side * NH + (n >> 1)) * P * LS + (n & 1);
+      const char* raw = nullptr;
+      if (n < N) {
+        const long long e0 = ((long long)b * N + n) * L + t0;
+        raw = (side ? cs_of(buf) : bs_of(buf)) + n * p.io_row + span_head(e0, si);
       }
-      bcn[e] = v;
+      for (int i = tid % 32; i < S; i += 32) {
+        const float v = (raw && i < cnt) ? to_f(reinterpret_cast<const TI*>(raw)[i]) : 0.0f;
+        dst[(i / J) * LS + 2 * (i % J)] = v;
+      }
     }
     __syncthreads();
 
-    if (active) {
+    {
       const TI* xr = reinterpret_cast<const TI*>(xs_of(buf) + c * p.x_row + span_head(myrow * Tx + xlo, si));
       const int hd = span_head(myrow * L + t0, si);
       char* dtrow = dts_of(buf) + c * p.io_row;  // the granule row: element 0 at byte hd
@@ -915,9 +923,10 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
       TO* yr = kInPlace ? reinterpret_cast<TO*>(dtrow + hd) : reinterpret_cast<TO*>(ys + c * p.y_row);
       const int i0 = lane * J;  // chunk-relative first token of this lane
 
-      // ---- per-token inputs of the lane's J tokens (identity (A,B) = (1,0) past the end)
-      float dl[J], du[J];
-      float2 yacc[J];
+      // ---- per-token inputs of the lane's J tokens (identity (a,b) = (1,0) past the end);
+      // delta and delta*u are kept duplicated, the form the paired FP32 instructions take
+      float2 dl2[J], du2[J], yacc[J];
+      float sdl = 0.0f;
       {
         float xw[J + 3];
 #pragma unroll
@@ -938,8 +947,10 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
           }
           const float v = valid ? to_f(dtr[i0 + jj]) + dtb : 0.0f;
           const float delta = valid ? (o.sp ? (kFast ? softplus_fast(v) : softplus(v)) : v) : 0.0f;
-          dl[jj] = delta;
-          du[jj] = valid ? delta * u : 0.0f;
+          const float dus = valid ? delta * u : 0.0f;
+          sdl += delta;
+          dl2[jj] = make_float2(delta, delta);
+          du2[jj] = make_float2(dus, dus);
           yacc[jj] = make_float2(dsk * u, 0.0f);
         }
       }
@@ -948,36 +959,42 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
 #pragma unroll 1
       for (int k = 0; k < NH; ++k) {
         const float2 A2 = *reinterpret_cast<const float2*>(a_s + c * NP + 2 * k);
-        float Bv0[J], Bv1[J];
+        const float* Bk = bcn + (k * P + lane) * LS;
+        const float* Ck = Bk + NH * P * LS;
+        // 1. the lane's decays and inputs, and its aggregate (Ar, Br) from a zero state;
+        //    Ar = exp2(A * sum(delta)) is the product of the decays, 0 across a reset
+        float2 a[J], bj[J];
+        float2 Br = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q = 0; q < J; q += 4) {
-          const float4 u0 = *reinterpret_cast<const float4*>(bcn + (2 * k) * S + i0 + q);
-          const float4 u1 = *reinterpret_cast<const float4*>(bcn + (2 * k + 1) * S + i0 + q);
-          Bv0[q] = u0.x; Bv0[q + 1] = u0.y; Bv0[q + 2] = u0.z; Bv0[q + 3] = u0.w;
-          Bv1[q] = u1.x; Bv1[q + 1] = u1.y; Bv1[q + 2] = u1.z; Bv1[q + 3] = u1.w;
-        }
-        // 1. the lane's decays and its aggregate from a zero state
-        float2 a[J];
-        float2 Ar = make_float2(1.f, 1.f), Br = make_float2(0.f, 0.f);
+        for (int q = 0; q < J; q += 2) {
+          const float4 u = *reinterpret_cast<const float4*>(Bk + 2 * q);
 #pragma unroll
-        for (int jj = 0; jj < J; ++jj) {
-          float2 aj = __fmul2_rn(make_float2(dl[jj], dl[jj]), A2);
-          aj.x = ex2(aj.x);
-          aj.y = ex2(aj.y);
-          if (jj == 0 && reset0) aj = make_float2(0.f, 0.f);
-          a[jj] = aj;
-          const float2 bj = __fmul2_rn(make_float2(Bv0[jj], Bv1[jj]), make_float2(du[jj], du[jj]));
-          Br = __ffma2_rn(aj, Br, bj);
-          Ar = __fmul2_rn(aj, Ar);
+          for (int e = 0; e < 2; ++e) {
+            const int jj = q + e;
+            float2 aj = __fmul2_rn(dl2[jj], A2);
+            aj.x = ex2(aj.x);
+            aj.y = ex2(aj.y);
+            if (jj == 0 && reset0) aj = make_float2(0.f, 0.f);
+            const float2 bv = e ? make_float2(u.z, u.w) : make_float2(u.x, u.y);
+            bj[jj] = __fmul2_rn(bv, du2[jj]);
+            Br = __ffma2_rn(aj, Br, bj[jj]);
+            a[jj] = aj;
+          }
         }
+        float2 Ar = __fmul2_rn(make_float2(sdl, sdl), A2);
+        Ar.x = reset0 ? 0.f : ex2(Ar.x);
+        Ar.y = reset0 ? 0.f : ex2(Ar.y);
         // 2. inclusive scan of the lanes' aggregates within the channel's P lanes
         float2 Ai = Ar, Bi = Br;
-        for (int off = 1; off < P; off <<= 1) {
-          const float2 Ap = make_float2(__shfl_up_sync(gmask, Ai.x, off, P), __shfl_up_sync(gmask, Ai.y, off, P));
-          const float2 Bp = make_float2(__shfl_up_sync(gmask, Bi.x, off, P), __shfl_up_sync(gmask, Bi.y, off, P));
-          if (lane >= off) {
-            Bi = __ffma2_rn(Ai, Bp, Bi);
-            Ai = __fmul2_rn(Ai, Ap);
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          if (off < P) {
+            const float2 Ap = make_float2(__shfl_up_sync(gmask, Ai.x, off, P), __shfl_up_sync(gmask, Ai.y, off, P));
+            const float2 Bp = make_float2(__shfl_up_sync(gmask, Bi.x, off, P), __shfl_up_sync(gmask, Bi.y, off, P));
+            if (lane >= off) {
+              Bi = __ffma2_rn(Ai, Bp, Bi);
+              Ai = __fmul2_rn(Ai, Ap);
+            }
           }
         }
         float2 Ae = make_float2(__shfl_up_sync(gmask, Ai.x, 1, P), __shfl_up_sync(gmask, Ai.y, 1, P));
@@ -990,20 +1007,14 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
         float2 h = __ffma2_rn(Ae, hc, Be);  // the state entering this lane's tokens
         __syncwarp(gmask);
         if (lane == P - 1) *reinterpret_cast<float2*>(carry + c * NP + 2 * k) = __ffma2_rn(Ai, hc, Bi);
-        // 3. replay from the entering state with the kept decays
-        float Cv0[J], Cv1[J];
+        // 3. replay from the entering state with the kept decays and inputs
 #pragma unroll
-        for (int q = 0; q < J; q += 4) {
-          const float4 u0 = *reinterpret_cast<const float4*>(bcn + (NP + 2 * k) * S + i0 + q);
-          const float4 u1 = *reinterpret_cast<const float4*>(bcn + (NP + 2 * k + 1) * S + i0 + q);
-          Cv0[q] = u0.x; Cv0[q + 1] = u0.y; Cv0[q + 2] = u0.z; Cv0[q + 3] = u0.w;
-          Cv1[q] = u1.x; Cv1[q + 1] = u1.y; Cv1[q + 2] = u1.z; Cv1[q + 3] = u1.w;
-        }
-#pragma unroll
-        for (int jj = 0; jj < J; ++jj) {
-          const float2 bj = __fmul2_rn(make_float2(Bv0[jj], Bv1[jj]), make_float2(du[jj], du[jj]));
-          h = __ffma2_rn(a[jj], h, bj);
-          yacc[jj] = __ffma2_rn(make_float2(Cv0[jj], Cv1[jj]), h, yacc[jj]);
+        for (int q = 0; q < J; q += 2) {
+          const float4 cv = *reinterpret_cast<const float4*>(Ck + 2 * q);
+          h = __ffma2_rn(a[q], h, bj[q]);
+          yacc[q] = __ffma2_rn(make_float2(cv.x, cv.y), h, yacc[q]);
+          h = __ffma2_rn(a[q + 1], h, bj[q + 1]);
+          yacc[q + 1] = __ffma2_rn(make_float2(cv.z, cv.w), h, yacc[q + 1]);
         }
       }
 #pragma unroll
@@ -1017,10 +1028,11 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
         }
         const int t = t0 + i;
         if (swap && t == 0) head_val = yo;
-        if (swap && t == L - 1)
-          yg[myrow * L] = from_f<TO>(yo);  // the tail output becomes the next head
-        else
+        if (swap && t == L - 1) {
+          if (active) yg[myrow * L] = from_f<TO>(yo);  // the tail output becomes the next head
+        } else {
           yr[i] = from_f<TO>(yo);
+        }
       }
       if (swap && t0 + cnt == L) {
         // token 0's output sits in lane 0; the lane that owns token L-1 stores it there
@@ -1028,13 +1040,13 @@ __global__ void __launch_bounds__(256) fwd_lanes_kernel(const FwdParams p) {
         if (lane == (cnt - 1) / J) yr[cnt - 1] = from_f<TO>(hv);
       }
       __syncwarp(gmask);
-      if (kInPlace && i0 < cnt) {  // each lane writes its own tokens back, 16-byte stores where aligned
+      if (kInPlace && active && i0 < cnt) {  // each lane writes its own tokens back, 16-byte stores where aligned
         const int off = hd + i0 * si;
         store_row<TO>(yg, myrow * L + t0 + i0, dtrow + (off & ~15), min(J, cnt - i0), swap && t0 + i0 == 0);
       }
       if (p.final_state && kc == nchunks - 1) {
         __syncwarp(gmask);
-        if (lane == 0) {
+        if (active && lane == 0) {
           float* fs = p.final_state + ((size_t)b * p.D + d) * N;
           for (int n = 0; n < N; ++n) fs[n] = carry[c * NP + n];
         }
@@ -1085,8 +1097,8 @@ int fwd_lanes_smem(const FwdParams& p, int si, int so, int NP) {
   s += (long long)p.d_tile * p.io_row * (gate ? 2 : 1);
   s += 2LL * p.N * p.io_row;
   s *= 2;                          // two staging buffers
-  s += 2LL * NP * p.chunk * 4;     // B, C in fp32
-  s += 2LL * p.d_tile * NP * 4;    // A * log2(e), carry
+  s += (long long)NP * p.lanes * (2 * kLaneTokens + 4) * 4;  // B, C in fp32, pair-interleaved
+  s += 2LL * p.d_tile * NP * 4;                               // A * log2(e), carry
   if (si != so) s += (long long)p.d_tile * p.y_row;
   return s > (1LL << 30) ? (1 << 30) : (int)s;
 }

@@ -48,7 +48,7 @@ struct FwdParams {
 constexpr int kModeChunk = 0;
 constexpr int kModeWhole = 1;
 constexpr int kModeLanes = 2;  // P lanes per channel split the tokens (warp-shuffle scan)
-constexpr int kLaneTokens = 16; // tokens per lane per chunk in kModeLanes
+constexpr int kLaneTokens = 16;  // tokens per lane per chunk in kModeLanes
 
 struct BwdParams {
   const void* u;

@@ -39,10 +39,13 @@ def divisors_upto(B, cap):
     return [v for v in (1, 2, 4, 8, 16, 32) if v <= cap and B % v == 0]
 
 
+LANE_TOKENS = 16  # tokens per lane per chunk in the library's lanes mode
+
+
 def candidates(B, T, D, N=16):
     """(B2, d_tile, chunk, lanes, chans_per_thread): one thread per channel or two side by
     side (lanes = 1) with whole-sample or chunked staging, and, for longer samples, P lanes
-    per channel (chunk = 8 P)."""
+    per channel (chunk = 16 P: each lane scans 16 tokens of a chunk)."""
     L = T + 2
     out = []
     tiles = [t for t in (32, 64, 128) if t <= max(32, ((D + 31) // 32) * 32)]
@@ -54,8 +57,8 @@ def candidates(B, T, D, N=16):
         out.append((B2, dt, ch, 1, cpt))
     if L >= 100:
         for B2, P, threads in itertools.product(divisors_upto(B, 4), (2, 4, 8, 16, 32), (64, 128, 256)):
-            if threads // P >= 1 and 8 * P <= 4 * L:
-                out.append((B2, threads // P, 8 * P, P, 1))
+            if threads // P >= 1 and LANE_TOKENS * P <= 4 * L:
+                out.append((B2, threads // P, LANE_TOKENS * P, P, 1))
     return out
 
 
