@@ -252,3 +252,118 @@ def mixer_layer_bwd(x, dt, z, Bm, Cm, A, Dskip, dt_bias, conv_w, conv_b, dout, *
     if db is not None:
         g["dconv_b"] = db
     return g
+
+
+# ---------------------------------------------------------------- ragged (variable-length) folding
+#
+# S samples of different lengths packed along time: sample s holds packed positions
+# [cu[s], cu[s+1]) of dt, z, Bm, Cm (rows [D, Ltot] and [N, Ltot]) and of the output; with
+# aux init its T_s = L_s - 2 patch tokens sit at x positions [cu[s] - 2s, cu[s+1] - 2s - 2).
+# The fold's reset and boundary-safe conv (techloop.online, Batch Folding with Periodic
+# State Reset and the convolution-boundary paragraph; sungsoo.github.io section 3.3) with
+# the fixed period replaced by the offsets.
+
+def _x_span(cu, s, aux):
+    a, e = int(cu[s]), int(cu[s + 1])
+    return (a - 2 * s, e - 2 * s - 2) if aux else (a, e)
+
+
+def mixer_layer_varlen(x, dt, z, Bm, Cm, A, Dskip, dt_bias, conv_w, conv_b, cu_seqlens, *, aux_init_in=False,
+                       swap_out=False, pad_left=None, dt_softplus=True, want_state=False):
+    """The ragged layer by its definition: every sample is mixer_layer run on its own slice.
+
+    Positions that belong to no sample stay 0.  Returns y [D, Ltot] (and the final states
+    [S, D, N] with want_state)."""
+    dt = _f64(dt)
+    D, Lt = dt.shape
+    cu = [int(v) for v in np.asarray(cu_seqlens).reshape(-1)]
+    S = len(cu) - 1
+    N = np.asarray(Bm).shape[0]
+    y = np.zeros((D, Lt))
+    fs = np.zeros((S, D, N))
+    xf, zf, Bf, Cf = _f64(x), _f64(z), _f64(Bm), _f64(Cm)
+    for s in range(S):
+        a, e = cu[s], cu[s + 1]
+        if e == a:
+            continue
+        xa, xe = _x_span(cu, s, aux_init_in)
+        res = mixer_layer(xf[None, :, xa:xe], dt[None, :, a:e], None if zf is None else zf[None, :, a:e],
+                          Bf[None, :, a:e], Cf[None, :, a:e], A, Dskip, dt_bias, conv_w, conv_b,
+                          aux_init_in=aux_init_in, swap_out=swap_out, pad_left=pad_left, dt_softplus=dt_softplus,
+                          want_state=want_state)
+        if want_state:
+            y[:, a:e], fs[s] = res[0][0], res[1][0]
+        else:
+            y[:, a:e] = res[0]
+    return (y, fs) if want_state else y
+
+
+def mixer_layer_packed_literal(x, dt, z, Bm, Cm, A, Dskip, dt_bias, conv_w, conv_b, cu_seqlens, *,
+                               aux_init_in=False, swap_out=False, pad_left=None, dt_softplus=True):
+    """The ragged fold read literally, written apart from the C routines: ONE recurrence
+    along each packed row with the transition Abar = 0 at every offset cu[s], conv taps
+    that read zero wherever they leave the sample of the tap's centre, aux tokens (the
+    mean of each sample's own x tokens) placed at every sample's ends, and each sample's
+    first and last outputs exchanged.  numpy fp64; small sizes only."""
+    dt, xf = _f64(dt), _f64(x)
+    D, Lt = dt.shape
+    cu = [int(v) for v in np.asarray(cu_seqlens).reshape(-1)]
+    S = len(cu) - 1
+    owner = np.full(Lt, -1)  # sample of each packed position, -1 for none
+    for s in range(S):
+        owner[cu[s]:cu[s + 1]] = s
+    # the conv input along the packed row (aux tokens filled in)
+    xa = np.zeros((D, Lt))
+    for s in range(S):
+        a, e = cu[s], cu[s + 1]
+        if e == a:
+            continue
+        if aux_init_in:
+            xs, xe = a - 2 * s, e - 2 * s - 2
+            m = xf[:, xs:xe].sum(axis=1) / (xe - xs)
+            xa[:, a], xa[:, e - 1] = m, m
+            xa[:, a + 1:e - 1] = xf[:, xs:xe]
+        else:
+            xa[:, a:e] = xf[:, a:e]
+    if conv_w is not None:
+        w = _f64(conv_w)
+        K = w.shape[1]
+        pl = (K - 1) // 2 if pad_left is None else pad_left
+        pre = np.zeros((D, Lt)) + (0.0 if conv_b is None else _f64(conv_b)[:, None])
+        for p in range(Lt):
+            for k in range(K):
+                q = p + k - pl
+                if 0 <= q < Lt and owner[q] == owner[p] and owner[p] >= 0:
+                    pre[:, p] += w[:, k] * xa[:, q]
+        u = pre / (1.0 + np.exp(-pre))
+    else:
+        u = xa
+    v = dt + (0.0 if dt_bias is None else _f64(dt_bias)[:, None])
+    if dt_softplus:
+        delta = np.where(v > 20.0, v, np.log1p(np.exp(np.minimum(v, 20.0))))
+    else:
+        delta = v
+    Af, Bf, Cf = _f64(A), _f64(Bm), _f64(Cm)
+    starts = set(cu[s] for s in range(S) if cu[s + 1] > cu[s])
+    h = np.zeros(Af.shape)  # [D, N]
+    y = np.zeros((D, Lt))
+    for p in range(Lt):
+        if owner[p] < 0:
+            h[:] = 0.0
+            continue
+        # the reset is a select, not a multiplication by 0, so nothing of the previous
+        # sample (not even inf or nan) enters this one
+        carried = np.zeros_like(h) if p in starts else np.exp(delta[:, p:p + 1] * Af) * h
+        h = carried + (delta[:, p] * u[:, p])[:, None] * Bf[None, :, p]
+        y[:, p] = h @ Cf[:, p]
+        if Dskip is not None:
+            y[:, p] += _f64(Dskip) * u[:, p]
+    if z is not None:
+        zf = _f64(z)
+        y = y * (zf / (1.0 + np.exp(-zf)))
+    if swap_out:
+        for s in range(S):
+            a, e = cu[s], cu[s + 1]
+            if e > a:
+                y[:, [a, e - 1]] = y[:, [e - 1, a]]
+    return y

@@ -28,18 +28,45 @@ MUTATIONS = {
 }
 
 
-@pytest.mark.parametrize("name", sorted(MUTATIONS))
-def test_pins_catch_planted_mistake(tmp_path, name):
-    src = open(os.path.join(ROOT, "oracle", "sfm_oracle.c")).read()
-    old, new = MUTATIONS[name]
+# mistakes in the ragged composition (oracle/__init__.py), caught by test_oracle_ragged_pins.py
+RAGGED_MUTATIONS = {
+    "ragged_x_offset": ("return (a - 2 * s, e - 2 * s - 2) if aux else (a, e)",
+                        "return (a - s, e - s - 2) if aux else (a, e)"),
+    "ragged_swap_dropped": ("aux_init_in=aux_init_in, swap_out=swap_out, pad_left=pad_left, dt_softplus=dt_softplus,\n"
+                            "                          want_state=want_state)",
+                            "aux_init_in=aux_init_in, swap_out=False, pad_left=pad_left, dt_softplus=dt_softplus,\n"
+                            "                          want_state=want_state)"),
+    "literal_no_reset": ("carried = np.zeros_like(h) if p in starts else np.exp(delta[:, p:p + 1] * Af) * h",
+                         "carried = np.exp(delta[:, p:p + 1] * Af) * h"),
+    "literal_conv_crosses_offsets": ("if 0 <= q < Lt and owner[q] == owner[p] and owner[p] >= 0:",
+                                     "if 0 <= q < Lt and owner[p] >= 0:"),
+    "literal_reset_multiplies": ("carried = np.zeros_like(h) if p in starts else np.exp(delta[:, p:p + 1] * Af) * h",
+                                 "carried = (0.0 if p in starts else np.exp(delta[:, p:p + 1] * Af)) * h"),
+}
+
+
+def _run_mutated(tmp_path, fname, old, new, pins, name):
+    src = open(os.path.join(ROOT, "oracle", fname)).read()
     assert src.count(old) >= 1, "mutation site moved: " + name
     work = tmp_path / "repo"
     shutil.copytree(os.path.join(ROOT, "oracle"), work / "oracle",
                     ignore=shutil.ignore_patterns("*.so", "__pycache__"))
-    (work / "oracle" / "sfm_oracle.c").write_text(src.replace(old, new, 1))
+    (work / "oracle" / fname).write_text(src.replace(old, new, 1))
     shutil.copytree(os.path.join(ROOT, "tests"), work / "tests",
                     ignore=shutil.ignore_patterns("__pycache__", "test_oracle_mutations.py"))
     os.symlink(os.path.join(ROOT, "selective_scan_sfm_b200"), work / "selective_scan_sfm_b200")
-    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider",
-                        "tests/test_oracle_pins.py"], cwd=work, capture_output=True, text=True, timeout=600)
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-p", "no:cacheprovider", pins], cwd=work,
+                       capture_output=True, text=True, timeout=600)
     assert r.returncode != 0, "planted mistake %s was not caught:\n%s" % (name, r.stdout[-2000:])
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(tmp_path, name):
+    old, new = MUTATIONS[name]
+    _run_mutated(tmp_path, "sfm_oracle.c", old, new, "tests/test_oracle_pins.py", name)
+
+
+@pytest.mark.parametrize("name", sorted(RAGGED_MUTATIONS))
+def test_ragged_pins_catch_planted_mistake(tmp_path, name):
+    old, new = RAGGED_MUTATIONS[name]
+    _run_mutated(tmp_path, "__init__.py", old, new, "tests/test_oracle_ragged_pins.py", name)
