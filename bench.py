@@ -51,7 +51,8 @@ def parse_args(argv=None):
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="stage4_t49")
     p.add_argument("--impl", default="sfm", choices=["sfm", "reference"])
-    p.add_argument("--no-extra", action="store_true", help="skip the T=196 line and the CPU baseline")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the T=196 and ragged lines and the CPU baseline")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-baseline sample budget")
     return p.parse_args(argv)
 
@@ -354,6 +355,92 @@ def measure(workload, steps, warmup, world, rank, device, seed_base=0, with_e2e=
     return res
 
 
+def ragged_algorithmic_bytes(S, D, Lt, N, K, in_size, out_size, aux=True):
+    """Bytes the ragged fused forward must move at least: x [D, Lt-2S], dt and z [D, Lt],
+    B and C [N, Lt], the offsets, the fp32 parameters; write y [D, Lt]."""
+    Lx = Lt - 2 * S if aux else Lt
+    acts = D * Lx * in_size + 2 * D * Lt * in_size + 2 * N * Lt * in_size
+    return acts + 4 * (S + 1) + D * (N + 3 + K) * 4 + D * Lt * out_size
+
+
+def _time_launches(launch, nsets, steps, warmup, world, device, stream):
+    import torch
+    for i in range(warmup):
+        launch(i)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        ev[i][0].record(stream)
+        launch(i)
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    if world > 1:
+        torch.distributed.barrier()
+    return t0.elapsed_time(t1), sum(a.elapsed_time(b) for a, b in ev) / steps
+
+
+def measure_ragged(steps, warmup, world, rank, device, seed_base=0, workload="ragged_t49_196"):
+    """The ragged forward on packed samples of unequal length, and, for comparison, the
+    fixed-layout forward on the same samples padded to the longest one (useful elements
+    counted in both)."""
+    import torch
+    from selective_scan_sfm_b200 import _abi, _scan_args, _varlen_args, synth
+
+    w = synth.WORKLOADS[workload]
+    S, D, N, K = w["S"], w["D"], w["N"], w["K"]
+    lens = synth.ragged_lengths(S, w["T_lo"], w["T_hi"], seed=seed_base)
+    Lt = sum(lens)
+    esz = 2 if w["dtype"] == "bf16" else 4
+    set_bytes = ragged_algorithmic_bytes(S, D, Lt, N, K, esz, esz)
+    nsets = max(2, math.ceil(2 * L2_BYTES / set_bytes) + 1)
+    stream = torch.cuda.current_stream(device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    lib = _abi.lib()
+    keep, cargs = [], []
+    for i in range(nsets):
+        d = synth.make_ragged_inputs(lens, D=D, N=N, K=K, dtype=w["dtype"], seed=seed_base + 31 * i)
+        dc = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+        a, y = _varlen_args(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], dc["cu_seqlens"], dc["z"], dc["Dskip"],
+                            dc["dt_bias"], dc["conv_w"], dc["conv_b"], None, None, 0, None, True, True, False, None)
+        keep.append((dc, y))
+        cargs.append((a, ctypes.c_void_p(dc["cu_seqlens"].data_ptr())))
+
+    def launch(i):
+        a, cu = cargs[i % nsets]
+        rc = lib.sfm_selective_scan_fold_varlen(ctypes.byref(a), cu, sp)
+        if rc != 0:
+            raise RuntimeError(_abi.status_string(rc))
+
+    total_ms, launch_ms = _time_launches(launch, nsets, steps, warmup, world, device, stream)
+    del keep, cargs
+    # the same samples padded to the longest one, fixed [S, D, Tmax + 2] layout
+    Tmax = max(lens) - 2
+    pb = synth.make_inputs(B=S, D=D, T=Tmax, N=N, K=K, dtype=w["dtype"], seed=seed_base + 7)
+    pbytes = algorithmic_bytes(S, D, Tmax, Tmax + 2, N, K, esz, esz)
+    psets = max(2, math.ceil(2 * L2_BYTES / pbytes) + 1)
+    pkeep, pargs = [], []
+    for i in range(psets):
+        dc = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in pb.items()}
+        a, y = _scan_args(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], dc["z"], dc["Dskip"], dc["dt_bias"],
+                          dc["conv_w"], dc["conv_b"], None, None, 0, None, True, True, False, None, 0, 0, 0)
+        pkeep.append((dc, y))
+        pargs.append(a)
+
+    def launch_padded(i):
+        rc = lib.sfm_selective_scan_fold(ctypes.byref(pargs[i % psets]), sp)
+        if rc != 0:
+            raise RuntimeError(_abi.status_string(rc))
+
+    ptotal_ms, plaunch_ms = _time_launches(launch_padded, psets, steps, warmup, world, device, stream)
+    return dict(total_ms=total_ms, avg_launch_ms=launch_ms, elements=D * Lt, bytes=set_bytes, w=w, lens=lens,
+                padded_total_ms=ptotal_ms, padded_launch_ms=plaunch_ms, padded_elements=S * D * (Tmax + 2))
+
+
 def max_over_ranks(v, world, device):
     if world == 1:
         return v
@@ -421,6 +508,24 @@ def main(argv=None):
                  "alu_frac": (r2["elements"] / (l2 * 1e-3)) / alu_peak_elems(w2["N"], w2["K"], 1965.0),
                  "B1": r2["variant"]["B1"]}
 
+    ragged = {}
+    if not args.no_extra:
+        rr = measure_ragged(args.steps, args.warmup, world, rank, device, seed_base=1000 * rank)
+        tr = max_over_ranks(rr["total_ms"], world, device)
+        lr = max_over_ranks(rr["avg_launch_ms"], world, device)
+        tp = max_over_ranks(rr["padded_total_ms"], world, device)
+        wr = rr["w"]
+        ragged = {"workload": "ragged_t49_196", "value": world * rr["elements"] * args.steps / (tr * 1e-3),
+                  "unit": "elems/s", "ms_per_step": tr / args.steps,
+                  "samples": wr["S"], "tokens": "T_s uniform on {%d..%d} + 2 aux, %d packed positions per rank"
+                  % (wr["T_lo"], wr["T_hi"], rr["elements"] // wr["D"]),
+                  "hbm": {"achieved": rr["bytes"] / (lr * 1e-3) / 1e9, "unit": "GB/s"},
+                  "alu_frac": (rr["elements"] / (lr * 1e-3)) / alu_peak_elems(wr["N"], wr["K"], 1965.0),
+                  "padded_fixed": {"value": world * rr["elements"] * args.steps / (tp * 1e-3), "unit": "elems/s",
+                                   "note": "useful elements/s of the fixed-layout forward on the same samples "
+                                           "padded to the longest (%d of %d elements useful)"
+                                           % (rr["elements"], rr["padded_elements"])}}
+
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -439,6 +544,8 @@ def main(argv=None):
     alu_peak = alu_peak_elems(w["N"], w["K"], sm_max)
     if extra:
         extra["hbm"].update(peak=hbm_peak, frac=extra["hbm"]["achieved"] / hbm_peak)
+    if ragged:
+        ragged["hbm"].update(peak=hbm_peak, frac=ragged["hbm"]["achieved"] / hbm_peak)
     cpu = None
     if not args.no_extra and world == 1:
         cpu = cpu_baseline(args.workload, args.cpu_seconds)
@@ -474,11 +581,13 @@ def main(argv=None):
         "kernel_ms": launch_ms,
         "e2e": {"value": e2e_value, "unit": "elems/s", "h2d_bytes_per_step": res["h2d"],
                 "d2h_bytes_per_step": res["d2h"]},
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps,  # timed region of the main workload: one kernel per step
         "clocks": ck,
     }
     if extra:
         line["t196"] = extra
+    if ragged:
+        line["ragged"] = ragged
     if cpu:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)

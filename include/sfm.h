@@ -172,6 +172,44 @@ typedef struct {
  */
 SFM_API sfm_status sfm_selective_scan_fold(const sfm_scan_args* args, sfm_stream_t stream);
 
+/*
+ * Ragged folding: the fused scan of sfm_selective_scan_fold over B samples of DIFFERENT
+ * lengths packed along time, with the state reset at every sample start given by an
+ * offset array instead of a fixed period.
+ *
+ *   cu_seqlens  DEVICE int32 [B+1]: sample s covers packed positions
+ *               [cu_seqlens[s], cu_seqlens[s+1]) (L_s = their difference tokens, aux
+ *               tokens included); normally 0 = cu_seqlens[0] <= ... <= cu_seqlens[B] = L.
+ *
+ * In `args`: B = number of samples, L = packed length (all samples' tokens), and the
+ * layouts are time-contiguous rows of the packed length:
+ *   x   [D, L - 2B] with aux_init (sample s at x offset cu_seqlens[s] - 2s, its T_s =
+ *       L_s - 2 patch tokens), else [D, L];
+ *   dt, z, y [D, L]; Bm, Cm [N, L]; final_state [B, D, N] (state after each sample).
+ * Every sample is computed exactly as sfm_selective_scan_fold computes one sample of
+ * length L_s: the conv sees zeros outside the sample, the aux tokens are the mean of the
+ * sample's own T_s tokens, the swap exchanges the sample's own first and last outputs.
+ * B1 (0 = look-up table at the mean length) groups B/B1 consecutive samples per folded
+ * row; reset_period must be 0; N <= 16; lanes must be 0 or 1 (one thread walks each
+ * channel, chunked staging).  y positions that belong to no sample are not written.
+ *
+ * The offsets are read on the device, so they are checked there: a sample whose offsets
+ * are out of order or outside [0, L] (or, with aux_init, shorter than 3 tokens or not
+ * matching x's packing) is skipped -- nothing of it is read or written -- and the
+ * device error word (sfm_get_device_error) is set to SFM_ERR_INVALID_ARG.  Everything
+ * else is validated on the host as for sfm_selective_scan_fold.
+ * Source: the fold with its per-sample reset and boundary-safe conv of
+ * techloop.online (Batch Folding with Periodic State Reset; the convolution-boundary
+ * paragraph) and sungsoo.github.io section 3.3, with the period replaced by offsets.
+ * Inputs of unequal length are the ones the pages point at beyond classification: the
+ * windowed detection backbones of the SF-Mamba repository (kd.iw.mk/sony/SF-Mamba, COCO
+ * Cascaded Mask-RCNN) and, in sungsoo.github.io's table of follow-up work, cameras or
+ * windows folded as one effective batch with their states kept apart.
+ */
+SFM_API sfm_status sfm_selective_scan_fold_varlen(const sfm_scan_args* args, const int* cu_seqlens,
+                                                  sfm_stream_t stream);
+
+
 /* Gradients produced by the scan backward (all fp32, caller-owned device memory). */
 typedef struct {
   uint32_t size;        /* sizeof(sfm_scan_grads)                                 */
@@ -294,7 +332,8 @@ SFM_API sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* o
 
 /*
  * Reads (and, if clear != 0, resets) the device-side error word that kernels set when
- * a bounded wait gives up.  Synchronises `stream` first.  *code = SFM_OK when clean.
+ * a bounded wait gives up (SFM_ERR_TIMEOUT) or ragged offsets are invalid
+ * (SFM_ERR_INVALID_ARG).  Synchronises `stream` first.  *code = SFM_OK when clean.
  */
 SFM_API sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code);
 

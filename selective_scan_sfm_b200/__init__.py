@@ -15,7 +15,7 @@ from . import _abi
 from ._abi import SFM_BF16, SFM_F32, SfmError
 
 __all__ = [
-    "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d", "sfm_selective_scan_fold",
+    "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d", "sfm_selective_scan_fold", "sfm_selective_scan_fold_varlen",
     "sfm_selective_scan_fold_bwd", "sfm_selective_scan_fold_bwd_noalloc", "sfm_mixer_bwd", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
     "SfmError", "library_path",
 ]
@@ -151,6 +151,71 @@ def sfm_selective_scan_fold(x, dt, Bm, Cm, A, *, z=None, Dskip=None, dt_bias=Non
                       dt_softplus, aux_init, swap_out, out_dtype, lanes, d_tile, chunk, exp2_split=exp2_split,
                       chans_per_thread=chans_per_thread)
     _abi.check(_abi.lib().sfm_selective_scan_fold(ctypes.byref(a), _stream(stream)), "sfm_selective_scan_fold")
+    return y
+
+
+def _varlen_args(x, dt, Bm, Cm, A, cu_seqlens, z, Dskip, dt_bias, conv_w, conv_b, y, final_state, B1, pad_left,
+                 dt_softplus, aux_init, swap_out, out_dtype, d_tile=0, chunk=0, exp2_split=0, chans_per_thread=0):
+    _dev(dt, "dt")
+    if dt.dim() != 2:
+        raise ValueError("dt must be [D, Ltot] (packed), got %s" % (tuple(dt.shape),))
+    D, Lt = dt.shape
+    io = dt.dtype
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 2:
+        raise ValueError("cu_seqlens must be [S+1] with S >= 1")
+    S = cu_seqlens.numel() - 1
+    _dev(x, "x", io, (D, Lt - 2 * S if aux_init else Lt))
+    N = Bm.shape[0] if isinstance(Bm, torch.Tensor) and Bm.dim() == 2 else -1
+    _dev(Bm, "Bm", io, (N, Lt))
+    _dev(Cm, "Cm", io, (N, Lt))
+    _dev(z, "z", io, (D, Lt), optional=True)
+    _dev(A, "A", torch.float32, (D, N))
+    _dev(Dskip, "Dskip", torch.float32, (D,), optional=True)
+    _dev(dt_bias, "dt_bias", torch.float32, (D,), optional=True)
+    K = 0
+    if conv_w is not None:
+        _dev(conv_w, "conv_w", torch.float32)
+        K = conv_w.shape[1]
+        _dev(conv_w, "conv_w", torch.float32, (D, K))
+    _dev(conv_b, "conv_b", torch.float32, (D,), optional=True)
+    od = io if out_dtype is None else out_dtype
+    if y is None:
+        y = torch.empty(D, Lt, dtype=od, device=dt.device)
+    _dev(y, "y", od, (D, Lt))
+    _dev(final_state, "final_state", torch.float32, (S, D, N), optional=True)
+    a = _abi.ScanArgs()
+    a.size = ctypes.sizeof(_abi.ScanArgs)
+    a.x, a.dt, a.z, a.Bm, a.Cm = (t.data_ptr() if t is not None else None for t in (x, dt, z, Bm, Cm))
+    a.A, a.Dskip, a.dt_bias, a.conv_w, a.conv_b = (t.data_ptr() if t is not None else None
+                                                   for t in (A, Dskip, dt_bias, conv_w, conv_b))
+    a.y = y.data_ptr()
+    a.final_state = final_state.data_ptr() if final_state is not None else None
+    a.B, a.D, a.L, a.N = S, D, Lt, N
+    a.K = K
+    a.pad_left = ((K - 1) // 2 if pad_left is None else int(pad_left)) if K else 0
+    a.B1 = int(B1)
+    a.reset_period = 0
+    a.dt_softplus, a.aux_init, a.swap_out = int(bool(dt_softplus)), int(bool(aux_init)), int(bool(swap_out))
+    a.in_dtype, a.out_dtype = _code(io), _code(od)
+    a.lanes, a.d_tile, a.chunk, a.exp2_split = 0, int(d_tile), int(chunk), int(exp2_split)
+    a.chans_per_thread = int(chans_per_thread)
+    return a, y
+
+
+def sfm_selective_scan_fold_varlen(x, dt, Bm, Cm, A, cu_seqlens, *, z=None, Dskip=None, dt_bias=None, conv_w=None,
+                                   conv_b=None, y=None, final_state=None, B1=0, pad_left=None, dt_softplus=True,
+                                   aux_init=False, swap_out=False, out_dtype=None, d_tile=0, chunk=0, exp2_split=0,
+                                   chans_per_thread=0, stream=None):
+    """Ragged fused forward: S samples of different lengths packed along time, the state
+    reset at every offset of cu_seqlens (int32 [S+1] on the device).  dt, z: [D, Ltot];
+    Bm, Cm: [N, Ltot]; x: [D, Ltot - 2S] with aux_init, else [D, Ltot]; final_state
+    [S, D, N].  Returns y [D, Ltot].  Offsets are checked on the device (see
+    sfm_get_device_error)."""
+    a, y = _varlen_args(x, dt, Bm, Cm, A, cu_seqlens, z, Dskip, dt_bias, conv_w, conv_b, y, final_state, B1, pad_left,
+                        dt_softplus, aux_init, swap_out, out_dtype, d_tile, chunk, exp2_split, chans_per_thread)
+    _abi.check(_abi.lib().sfm_selective_scan_fold_varlen(ctypes.byref(a), ctypes.c_void_p(cu_seqlens.data_ptr()),
+                                                         _stream(stream)), "sfm_selective_scan_fold_varlen")
     return y
 
 

@@ -19,7 +19,7 @@ ENTRY_POINTS = (
     "sfm_status_string", "sfm_abi_version", "sfm_last_cuda_error", "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d",
     "sfm_selective_scan_fold", "sfm_scan_bwd_workspace_size", "sfm_selective_scan_fold_bwd",
     "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error", "sfm_selective_scan_fold_bwd_noalloc",
-    "sfm_mixer_bwd_workspace_size", "sfm_mixer_bwd",
+    "sfm_mixer_bwd_workspace_size", "sfm_mixer_bwd", "sfm_selective_scan_fold_varlen",
 )
 
 #: Size of the workspace built into the library for sfm_selective_scan_fold_bwd_noalloc.

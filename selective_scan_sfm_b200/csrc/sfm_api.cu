@@ -4,6 +4,7 @@
 // Validation is complete before any CUDA call, so every argument error returns
 // synchronously and leaves the device untouched.  The library keeps no mutable state
 // besides the once-per-kernel shared-memory attribute and the device error word.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdlib>
@@ -144,6 +145,42 @@ sfm_status validate_scan(const sfm_scan_args* a, bool bwd) {
         overlaps(a->y, ybytes, a->Cm, bcbytes))
       return SFM_ERR_INVALID_ARG;
   }
+  return SFM_OK;
+}
+
+// The ragged forward: B samples packed along time in rows of L (the packed total)
+// positions; the per-sample offsets live on the device and are checked by the kernel.
+sfm_status validate_varlen(const sfm_scan_args* a, const int* cu_seqlens) {
+  if (!a || a->size != sizeof(sfm_scan_args) || !cu_seqlens) return SFM_ERR_INVALID_ARG;
+  if (!a->x || !a->dt || !a->Bm || !a->Cm || !a->A || !a->y) return SFM_ERR_INVALID_ARG;
+  if (a->B < 1 || a->D < 1 || a->L < 1 || a->N < 1) return SFM_ERR_INVALID_ARG;
+  if (a->N > kMaxNFused) return SFM_ERR_UNSUPPORTED;
+  if ((a->dt_softplus | a->aux_init | a->swap_out) & ~1) return SFM_ERR_INVALID_ARG;
+  if (a->aux_init && (long long)a->L < 3LL * a->B) return SFM_ERR_INVALID_ARG;  // >= 3 tokens per sample
+  if (a->conv_w && (a->K < 1 || a->K > SFM_MAX_K || a->pad_left < 0 || a->pad_left >= a->K))
+    return SFM_ERR_INVALID_ARG;
+  if (a->B1 < 0 || (a->B1 > 0 && a->B % a->B1 != 0)) return SFM_ERR_INVALID_ARG;
+  if (a->B1 > kMaxB1) return SFM_ERR_UNSUPPORTED;
+  if (a->reset_period != 0) return SFM_ERR_UNSUPPORTED;  // the resets follow cu_seqlens
+  if (!dtype_ok(a->in_dtype) || !dtype_ok(a->out_dtype)) return SFM_ERR_INVALID_ARG;
+  if (a->in_dtype == SFM_F32 && a->out_dtype == SFM_BF16) return SFM_ERR_UNSUPPORTED;
+  if (a->lanes > 1) return SFM_ERR_UNSUPPORTED;  // one thread walks each channel
+  if (a->lanes < 0 || a->d_tile < 0 || a->d_tile > kMaxDTile) return SFM_ERR_UNSUPPORTED;
+  if (a->chunk < 0 || a->chunk > kMaxChunk || (a->chunk % 8) != 0) return SFM_ERR_UNSUPPORTED;
+  if (a->exp2_split < 0 || a->exp2_split > 4) return SFM_ERR_UNSUPPORTED;
+  if (a->chans_per_thread < 0 || a->chans_per_thread > 2) return SFM_ERR_UNSUPPORTED;
+  const void* acts[] = {a->x, a->dt, a->z, a->Bm, a->Cm, a->y};
+  for (const void* p : acts)
+    if (p && !aligned16(p)) return SFM_ERR_MISALIGNED;
+  if (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) return SFM_ERR_MISALIGNED;
+  const long long si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);
+  const long long dl = (long long)a->D * a->L;
+  const long long xbytes = (long long)a->D * (a->aux_init ? a->L - 2LL * a->B : a->L) * si;
+  const long long bcbytes = (long long)a->N * a->L * si, ybytes = dl * so;
+  if (overlaps(a->y, ybytes, a->x, xbytes) || overlaps(a->y, ybytes, a->dt, dl * si) ||
+      overlaps(a->y, ybytes, a->z, dl * si) || overlaps(a->y, ybytes, a->Bm, bcbytes) ||
+      overlaps(a->y, ybytes, a->Cm, bcbytes) || overlaps(a->y, ybytes, cu_seqlens, 4LL * (a->B + 1)))
+    return SFM_ERR_INVALID_ARG;
   return SFM_OK;
 }
 
@@ -329,6 +366,11 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
   p.L = a->L;
   p.N = a->N;
   p.Tx = a->aux_init ? a->L - 2 : a->L;
+  p.x_cs = p.Tx;
+  p.io_cs = p.bc_cs = a->L;
+  p.x_elems = (long long)a->B * a->D * p.Tx;
+  p.io_elems = (long long)a->B * a->D * a->L;
+  p.bc_elems = (long long)a->B * a->N * a->L;
   p.K = a->conv_w ? a->K : 1;
   p.pad_left = a->conv_w ? a->pad_left : 0;
   p.B2 = a->B / (a->B1 ? a->B1 : v.B1);
@@ -413,6 +455,73 @@ sfm_status sfm_selective_scan_fold(const sfm_scan_args* a, sfm_stream_t stream) 
       if (p.smem_bytes > fwd_max_smem()) return SFM_ERR_UNSUPPORTED;
     }
   }
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_fwd(p, a->in_dtype, a->out_dtype, NP, stream));
+}
+
+sfm_status sfm_selective_scan_fold_varlen(const sfm_scan_args* a, const int* cu_seqlens, sfm_stream_t stream) {
+  sfm_status st = validate_varlen(a, cu_seqlens);
+  if (st != SFM_OK) return st;
+  // the launch shape of the look-up table at the mean sample length, in chunked mode
+  const int Lmean = (int)std::max(1LL, (long long)a->L / a->B);
+  const int Tmean = std::max(1, a->aux_init ? Lmean - 2 : Lmean);
+  const sfm_variant v = choose(a->B, Tmean, a->D, a->N);
+  FwdParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.x = a->x;
+  p.dt = a->dt;
+  p.z = a->z;
+  p.Bm = a->Bm;
+  p.Cm = a->Cm;
+  p.A = a->A;
+  p.Dskip = a->Dskip;
+  p.dt_bias = a->dt_bias;
+  p.conv_w = a->conv_w;
+  p.conv_b = a->conv_b;
+  p.y = a->y;
+  p.final_state = a->final_state;
+  p.cu_seqlens = cu_seqlens;
+  p.B = a->B;
+  p.D = a->D;
+  p.L = a->L;
+  p.N = a->N;
+  p.Tx = a->aux_init ? a->L - 2 * a->B : a->L;
+  p.x_cs = p.Tx;
+  p.io_cs = p.bc_cs = a->L;
+  p.x_elems = (long long)a->D * p.Tx;
+  p.io_elems = (long long)a->D * a->L;
+  p.bc_elems = (long long)a->N * a->L;
+  p.K = a->conv_w ? a->K : 1;
+  p.pad_left = a->conv_w ? a->pad_left : 0;
+  p.B2 = a->B / (a->B1 ? a->B1 : v.B1);
+  const bool lut_chunked = v.lanes == 1;
+  p.d_tile = a->d_tile ? a->d_tile : (lut_chunked ? v.d_tile : 64);
+  // samples of unequal length: chunks of 32..64 tokens measured best (fewer steps per sample
+  // than the fixed layout's short chunks, little waste in each sample's last chunk)
+  p.chunk = a->chunk ? a->chunk : (lut_chunked ? std::max(32, std::min(v.chunk, 64)) : 64);
+  p.exp2_fma_pairs = a->exp2_split ? a->exp2_split - 1 : v.exp2_pairs;
+  p.cpt = a->chans_per_thread ? a->chans_per_thread : ((a->d_tile || a->chunk || !lut_chunked) ? 1 : v.chans_per_thread);
+  if (p.cpt == 2 && !(a->conv_w && a->z && a->dt_softplus && a->K == 4 && a->N > 8 && a->N <= 16 &&
+                      a->D % 2 == 0 && p.d_tile % 2 == 0))
+    p.cpt = 1;
+  p.flags = (a->dt_softplus ? kSoftplus : 0) | (a->aux_init ? kAuxInit : 0) | (a->swap_out ? kSwapOut : 0) |
+            (a->conv_w ? kConv : 0) | (a->z ? kGate : 0);
+  const int si = esize_of(a->in_dtype), so = esize_of(a->out_dtype);
+  int NP = 2;
+  while (NP < a->N) NP <<= 1;
+  p.np = NP;
+  if (a->B / p.B2 > kMaxB1) return SFM_ERR_UNSUPPORTED;
+  p.mode = kModeChunk;
+  p.lanes = 1;
+  p.x_row = fwd_x_row(p.chunk, 4, si);
+  p.io_row = fwd_io_row(p.chunk, si);
+  p.y_row = fwd_y_row(p.chunk, so);
+  p.smem_bytes = fwd_chunk_smem(p, si, so, NP);
+  while (p.smem_bytes > fwd_max_smem() && !a->d_tile && p.d_tile > 32) {
+    p.d_tile /= 2;
+    p.smem_bytes = fwd_chunk_smem(p, si, so, NP);
+  }
+  if (p.smem_bytes > fwd_max_smem()) return SFM_ERR_UNSUPPORTED;
   if (fault_injected()) return SFM_ERR_CUDA;
   return cuda_status(launch_fwd(p, a->in_dtype, a->out_dtype, NP, stream));
 }

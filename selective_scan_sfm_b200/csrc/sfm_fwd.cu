@@ -593,6 +593,12 @@ __global__ void __launch_bounds__(128) fwd_whole_kernel(const FwdParams p) {
 // copies of step s+1 (the next chunk, or the first chunk of the next sample of the folded
 // row) are in flight.  Buffer layout per stage: [x rows][dt rows][z rows][B rows][C rows];
 // after both stages: [bct][y rows if not in place].
+//
+// The samples of a folded row are either the fixed [B,D,L] layout (sample s at element
+// s*D*L, every sample L long) or the ragged packed layout (sample s at packed offset
+// cu_seqlens[s] of rows that are the packed length long, its own length
+// cu_seqlens[s+1] - cu_seqlens[s]); in both the state restarts at each sample's first
+// token and the conv never reads across a sample boundary.
 template <typename TI, typename TO, int NH, bool STD, int PE, int CPT>
 __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
   constexpr bool kInPlace = std::is_same<TI, TO>::value;
@@ -604,13 +610,13 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
   const int lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
   const int d0 = blockIdx.x * p.d_tile;
   const int dcount = min(p.d_tile, p.D - d0);
-  const int b1 = blockIdx.y;
   const int c0 = tid * CPT;
   const bool active = c0 < dcount;
-  const int L = p.L, N = p.N, S = p.chunk, Tx = p.Tx;
-  const Opts o = make_opts(p);
+  const int N = p.N, S = p.chunk;
+  Opts o = make_opts(p);  // o.L and o.Tx follow the sample being walked
   const bool swap = p.flags & kSwapOut;
   const int K = o.conv ? o.K : 1, pl = o.pl;
+  const int s0 = blockIdx.y * p.B2, ns = min(p.B2, p.B - s0);  // this folded row's samples
 
   const int stage_bytes = p.d_tile * p.x_row + p.d_tile * p.io_row * (o.gate ? 2 : 1) + 2 * N * p.io_row;
   float* bct = reinterpret_cast<float*>(smem + 2 * stage_bytes);
@@ -625,44 +631,82 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
 #pragma unroll
   for (int ch = 0; ch < CPT; ++ch) load_chan(c[ch], p, d0 + (active ? c0 + ch : 0), o.conv);
 
-  const long long x_bytes = (long long)p.B * p.D * Tx * si;
-  const long long io_bytes = (long long)p.B * p.D * L * si;
-  const long long bc_bytes = (long long)p.B * N * L * si;
+  const long long x_bytes = p.x_elems * si, io_bytes = p.io_elems * si, bc_bytes = p.bc_elems * si;
   const char* xg = static_cast<const char*>(p.x);
   const char* dtg = static_cast<const char*>(p.dt);
   const char* zg = static_cast<const char*>(p.z);
   const char* bg = static_cast<const char*>(p.Bm);
   const char* cg = static_cast<const char*>(p.Cm);
   TO* yg = static_cast<TO*>(p.y);
-  const int nchunks = (L + S - 1) / S;
-  const int nsteps = p.B2 * nchunks;
+
+  // One step = chunk kc of sample s0 + j.  len/tx: the sample's tokens (with aux) and x
+  // tokens; xb, ib, bb: element offsets of its channel-0 x row, channel-0 dt/z/y row and
+  // state-0 B/C row.  A sample with len 0 has no steps.
+  struct Step {
+    int j, kc, len, tx;
+    long long xb, ib, bb;
+  };
+  auto load_sample = [&](Step& q) {
+    const int s = s0 + q.j;
+    if (!p.cu_seqlens) {
+      q.len = p.L;
+      q.tx = p.Tx;
+      q.xb = (long long)s * p.D * p.Tx;
+      q.ib = (long long)s * p.D * p.L;
+      q.bb = (long long)s * N * p.L;
+      return;
+    }
+    const int a = p.cu_seqlens[s], e = p.cu_seqlens[s + 1];
+    // offsets out of order or out of the packed rows, or an aux sample without a patch
+    // token: reported in the device error word; the sample is skipped, nothing is read
+    const bool bad = a < 0 || e < a || e > p.L ||
+                     (o.aux && (e - a < 3 || a - 2LL * s < 0 || e - 2LL * s - 2 > p.Tx));
+    if (bad) {
+      if (tid == 0) atomicExch(&g_device_error, (unsigned)SFM_ERR_INVALID_ARG);
+      q.len = 0;
+      return;
+    }
+    q.len = e - a;
+    q.tx = o.aux ? q.len - 2 : q.len;
+    q.xb = o.aux ? a - 2LL * s : a;
+    q.ib = a;
+    q.bb = a;
+  };
+  // moves q to the first step at or after (q.j, q.kc) that has tokens
+  auto settle = [&](Step& q) {
+    while (q.j < ns) {
+      if (q.kc == 0) load_sample(q);
+      if (q.kc * S < q.len) return;
+      ++q.j;
+      q.kc = 0;
+    }
+  };
 
   // x tokens a chunk needs: xa positions [t0-pl, t0+cnt-1+K-1-pl], clamped to the sample
-  auto x_window = [&](int t0, int cnt, int& xlo, int& xhi) {
+  auto x_window = [&](int t0, int cnt, int tx, int& xlo, int& xhi) {
     const int slo = t0 - pl - o.off, shi = t0 + cnt - 1 + (K - 1 - pl) - o.off;
     xlo = max(slo, 0);
-    xhi = min(shi + 1, Tx);
+    xhi = min(shi + 1, tx);
   };
-  // issues the copies of step `st` into buffer `buf` (each thread its own rows; threads
+  // issues the copies of step q into buffer `buf` (each thread its own rows; threads
   // 0..2N-1 the B and C rows) and commits them as one group
-  auto stage = [&](int st, int buf) {
-    const int b = b1 * p.B2 + st / nchunks, t0 = (st % nchunks) * S, cnt = min(S, L - t0);
-    const long long row0 = (long long)b * p.D + d0;
+  auto stage = [&](const Step& q, int buf) {
+    const int t0 = q.kc * S, cnt = min(S, q.len - t0);
     int xlo, xhi;
-    x_window(t0, cnt, xlo, xhi);
+    x_window(t0, cnt, q.tx, xlo, xhi);
     if (active) {
 #pragma unroll
       for (int ch = 0; ch < CPT; ++ch) {
-        const long long myrow = row0 + c0 + ch;
         const int r = c0 + ch;
-        copy_span_async(xs_of(buf) + r * p.x_row, xg, myrow * Tx + xlo, xhi - xlo, si, x_bytes, 0, 1);
-        copy_span_async(dts_of(buf) + r * p.io_row, dtg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
-        if (o.gate) copy_span_async(zs_of(buf) + r * p.io_row, zg, myrow * L + t0, cnt, si, io_bytes, 0, 1);
+        const long long xrow = q.xb + (d0 + r) * p.x_cs, iorow = q.ib + (d0 + r) * p.io_cs;
+        copy_span_async(xs_of(buf) + r * p.x_row, xg, xrow + xlo, xhi - xlo, si, x_bytes, 0, 1);
+        copy_span_async(dts_of(buf) + r * p.io_row, dtg, iorow + t0, cnt, si, io_bytes, 0, 1);
+        if (o.gate) copy_span_async(zs_of(buf) + r * p.io_row, zg, iorow + t0, cnt, si, io_bytes, 0, 1);
       }
     }
     for (int r = tid; r < 2 * N; r += nthr) {
       const int n = r % N;
-      const long long e0 = ((long long)b * N + n) * L + t0;
+      const long long e0 = q.bb + n * p.bc_cs + t0;
       copy_span_async((r < N ? bs_of(buf) : cs_of(buf)) + n * p.io_row, r < N ? bg : cg, e0, cnt, si, bc_bytes, 0,
                       1);
     }
@@ -670,34 +714,41 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
   };
 
   TO head_val[CPT];
-  stage(0, 0);
-  for (int st = 0; st < nsteps; ++st) {
-    const int buf = st & 1;
-    const int j = st / nchunks, kc = st % nchunks;
-    const int b = b1 * p.B2 + j;
-    const long long row0 = (long long)b * p.D + d0;
-    const int t0 = kc * S, cnt = min(S, L - t0);
+  Step cur{0, 0, 0, 0, 0, 0, 0};
+  settle(cur);
+  if (cur.j < ns) stage(cur, 0);
+  for (int it = 0; cur.j < ns; ++it) {
+    const int buf = it & 1;
+    Step nxt = cur;
+    ++nxt.kc;
+    settle(nxt);
+    const int s = s0 + cur.j, kc = cur.kc;
+    const int t0 = kc * S, cnt = min(S, cur.len - t0);
+    const bool last = t0 + cnt == cur.len;
+    o.L = cur.len;
+    o.Tx = cur.tx;
     int xlo, xhi;
-    x_window(t0, cnt, xlo, xhi);
+    x_window(t0, cnt, cur.tx, xlo, xhi);
     if (kc == 0) {  // a new sample: the state restarts; the aux mean needs the whole x row
 #pragma unroll
       for (int ch = 0; ch < CPT; ++ch) {
-        c[ch].mean =
-            (o.aux && active) ? row_mean(reinterpret_cast<const TI*>(xg) + (row0 + c0 + ch) * Tx, Tx) : 0.0f;
+        c[ch].mean = (o.aux && active) ? row_mean(reinterpret_cast<const TI*>(xg) + cur.xb +
+                                                      (d0 + c0 + ch) * p.x_cs, cur.tx)
+                                       : 0.0f;
 #pragma unroll
         for (int k = 0; k < NH; ++k) c[ch].h[k] = make_float2(0.f, 0.f);
       }
     }
-    if (st + 1 < nsteps) {
-      stage(st + 1, buf ^ 1);
+    if (nxt.j < ns) {
+      stage(nxt, buf ^ 1);
       cp_async_wait<1>();  // this step's group has landed; the next one stays in flight
     } else {
       cp_async_wait<0>();
     }
     __syncthreads();
 
-    transpose_bc<TI, NH>(bct, bs_of(buf), cs_of(buf), p.io_row, (unsigned)((long long)b * N * L + t0), (unsigned)L,
-                         N, cnt, tid, nthr, true);
+    transpose_bc<TI, NH>(bct, bs_of(buf), cs_of(buf), p.io_row, (unsigned)(cur.bb + t0), (unsigned)p.bc_cs, N, cnt,
+                         tid, nthr, true);
     __syncthreads();
 
     if (active) {
@@ -707,10 +758,10 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
       TO* yr[CPT];
 #pragma unroll
       for (int ch = 0; ch < CPT; ++ch) {
-        const long long myrow = row0 + c0 + ch;
         const int r = c0 + ch;
-        xr[ch] = reinterpret_cast<const TI*>(xs_of(buf) + r * p.x_row + span_head(myrow * Tx + xlo, si));
-        const int hd = span_head(myrow * L + t0, si);
+        const long long xrow = cur.xb + (d0 + r) * p.x_cs, iorow = cur.ib + (d0 + r) * p.io_cs;
+        xr[ch] = reinterpret_cast<const TI*>(xs_of(buf) + r * p.x_row + span_head(xrow + xlo, si));
+        const int hd = span_head(iorow + t0, si);
         dtr[ch] = reinterpret_cast<const TI*>(dts_of(buf) + r * p.io_row + hd);
         zr[ch] = o.gate ? reinterpret_cast<const TI*>(zs_of(buf) + r * p.io_row + hd) : dtr[ch];
         yr[ch] = kInPlace ? reinterpret_cast<TO*>(dts_of(buf) + r * p.io_row + hd)
@@ -720,9 +771,9 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
       if (swap) {
 #pragma unroll
         for (int ch = 0; ch < CPT; ++ch) {
-          if (t0 == 0) head_val[ch] = yr[ch][0];  // goes to position L-1
-          if (t0 + cnt == L) {
-            yg[(row0 + c0 + ch) * L] = yr[ch][cnt - 1];  // the tail output becomes the next head
+          if (t0 == 0) head_val[ch] = yr[ch][0];  // goes to the sample's last position
+          if (last) {
+            yg[cur.ib + (d0 + c0 + ch) * p.io_cs] = yr[ch][cnt - 1];  // the tail output becomes the next head
             yr[ch][cnt - 1] = head_val[ch];
           }
         }
@@ -731,11 +782,12 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
       if (kInPlace)
 #pragma unroll
         for (int ch = 0; ch < CPT; ++ch)
-          store_row<TO>(yg, (row0 + c0 + ch) * L + t0, dts_of(buf) + (c0 + ch) * p.io_row, cnt, swap && t0 == 0);
-      if (p.final_state && kc == nchunks - 1) {
+          store_row<TO>(yg, cur.ib + (d0 + c0 + ch) * p.io_cs + t0, dts_of(buf) + (c0 + ch) * p.io_row, cnt,
+                        swap && t0 == 0);
+      if (p.final_state && last) {
 #pragma unroll
         for (int ch = 0; ch < CPT; ++ch) {
-          float* fs = p.final_state + ((size_t)b * p.D + d0 + c0 + ch) * N;
+          float* fs = p.final_state + ((size_t)s * p.D + d0 + c0 + ch) * N;
 #pragma unroll
           for (int k = 0; k < NH; ++k) {
             if (2 * k < N) fs[2 * k] = c[ch].h[k].x;
@@ -744,16 +796,17 @@ __global__ void __launch_bounds__(128) fwd_chunk_kernel(const FwdParams p) {
         }
       }
     }
-    __syncthreads();  // the buffer of this step is free for the copies of step st + 2
+    __syncthreads();  // the buffer of this step is free for the copies of step it + 2
     if (!kInPlace) {  // separate output rows: coalesced element stores by rows
       for (int r = warp; r < dcount; r += nwarps) {
         const char* src = ys + r * p.y_row;
-        TO* dst = yg + (row0 + r) * L + t0;
+        TO* dst = yg + cur.ib + (d0 + r) * p.io_cs + t0;
         for (int i = lane; i < cnt; i += 32)
           if (!(swap && t0 + i == 0)) dst[i] = *reinterpret_cast<const TO*>(src + i * so);
       }
       __syncthreads();  // ys is rewritten by the next step's walk
     }
+    cur = nxt;
   }
 }
 

@@ -30,6 +30,12 @@ struct FwdParams {
   void* y;
   float* final_state;
   int B, D, L, N, Tx;  // Tx = tokens per row of x (L-2 with aux init, else L)
+  // Ragged layout (chunked mode only): B samples packed along time, sample s at packed
+  // positions [cu_seqlens[s], cu_seqlens[s+1]); L and Tx are then the packed totals.
+  // NULL for the fixed [B,D,L] layout.
+  const int* cu_seqlens;
+  long long x_cs, io_cs, bc_cs;           // elements between channel rows (x; dt, z, y) and state rows (B, C)
+  long long x_elems, io_elems, bc_elems;  // elements of x, of each of dt/z/y, of each of B/C
   int K, pad_left;
   int B2;              // samples walked by one CTA (samples per folded row)
   int d_tile;          // channels per CTA (= threads per CTA for one lane per channel)

@@ -29,6 +29,9 @@ WORKLOADS = {
     "stage3_t196": dict(B=128, D=640, T=196, N=16, K=4, dtype="bf16"),
     # longer sequences (28x28 tokens) where folding matters less
     "long_t784": dict(B=16, D=320, T=784, N=16, K=4, dtype="bf16"),
+    # ragged batch: 128 samples of 49..196 patch tokens (windowed / detection-like mix of
+    # the stage-4 and stage-3 token counts) packed along time, stage-3 channels
+    "ragged_t49_196": dict(S=128, T_lo=49, T_hi=196, D=640, N=16, K=4, dtype="bf16", ragged=True),
     # four mixer layers in a chain at the stage-3 shape
     "chain4_stage3": dict(B=64, D=640, T=196, N=16, K=4, dtype="bf16", layers=4),
 }
@@ -66,6 +69,45 @@ def make_inputs(B: int, D: int, T: int, N: int, K: int = 4, dtype: str = "bf16",
     return dict(x=x.to(io), z=z.to(io), dt=dt.to(io), Bm=Bm.to(io), Cm=Cm.to(io),
                 A=A.contiguous(), Dskip=Dskip, dt_bias=dt_bias, conv_w=conv_w.contiguous(),
                 conv_b=conv_b, B=B, D=D, T=T, L=L, N=N, K=K, dtype=dtype)
+
+
+def ragged_lengths(S: int, T_lo: int, T_hi: int, seed: int = 0, aux: bool = True) -> list:
+    """Per-sample token counts L_s for a ragged batch: T_s uniform on {T_lo..T_hi} patch
+    tokens (plus the two aux tokens with ``aux``)."""
+    g = torch.Generator().manual_seed(int(seed) + 991)
+    T = torch.randint(T_lo, T_hi + 1, (S,), generator=g)
+    return [int(t) + (2 if aux else 0) for t in T]
+
+
+def make_ragged_inputs(lens, D: int, N: int, K: int = 4, dtype: str = "bf16", seed: int = 0,
+                       random_A: bool = False, aux: bool = True) -> dict:
+    """One layer's inputs for S samples of lengths ``lens`` (tokens per sample, aux tokens
+    included) packed along time, drawn like ``make_inputs``: x [D, Ltot - 2S] with ``aux``
+    (else [D, Ltot]), z and dt [D, Ltot], Bm and Cm [N, Ltot], cu_seqlens int32 [S+1]."""
+    g = torch.Generator().manual_seed(int(seed))
+    S = len(lens)
+    cu = [0]
+    for n in lens:
+        cu.append(cu[-1] + int(n))
+    Lt = cu[-1]
+    io = _TORCH_DT[dtype]
+    x = torch.randn(D, Lt - 2 * S if aux else Lt, generator=g)
+    z = torch.randn(D, Lt, generator=g)
+    dt = 0.5 * torch.randn(D, Lt, generator=g)
+    u01 = torch.rand(D, generator=g, dtype=torch.float64)
+    dt_bias = torch.log(torch.expm1(1e-3 + u01 * (1e-1 - 1e-3))).float()
+    Bm = torch.randn(N, Lt, generator=g)
+    Cm = torch.randn(N, Lt, generator=g)
+    Dskip = torch.randn(D, generator=g)
+    conv_w = torch.rand(D, K, generator=g) - 0.5
+    conv_b = torch.rand(D, generator=g) - 0.5
+    if random_A:
+        A = -torch.exp(torch.randn(D, N, generator=g))
+    else:
+        A = -torch.arange(1, N + 1, dtype=torch.float32).repeat(D, 1)
+    return dict(x=x.to(io), z=z.to(io), dt=dt.to(io), Bm=Bm.to(io), Cm=Cm.to(io), A=A.contiguous(), Dskip=Dskip,
+                dt_bias=dt_bias, conv_w=conv_w.contiguous(), conv_b=conv_b,
+                cu_seqlens=torch.tensor(cu, dtype=torch.int32), S=S, D=D, Ltot=Lt, N=N, K=K, dtype=dtype)
 
 
 def make_chain(B: int, D: int, T: int, N: int, layers: int = 4, K: int = 4, dtype: str = "bf16",
