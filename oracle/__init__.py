@@ -367,3 +367,25 @@ def mixer_layer_packed_literal(x, dt, z, Bm, Cm, A, Dskip, dt_bias, conv_w, conv
             if e > a:
                 y[:, [a, e - 1]] = y[:, [e - 1, a]]
     return y
+
+
+# ---------------------------------------------------------------- per-token projections
+#
+# The dense maps around the scan (the Mamba block's input, state and step-size
+# projections; background of sungsoo.github.io, Sources and Evidence Notes, items 4-5):
+# P[m, n] = sum_k W[m, k] X[n, k] over tokens n = b*L + t.
+
+def proj(W, X, L, M0=None, token_major=False):
+    """P = W X^T in fp64 (numpy matmul), laid out as the projection kernel writes it:
+    token-major [Ntok, M], or channel-major ([B, M0, L], [B, M - M0, L]) with rows split
+    at M0 (the second part None when M0 == M)."""
+    W, X = _f64(W), _f64(X)
+    M = W.shape[0]
+    Ntok = X.shape[0]
+    P = W @ X.T  # [M, Ntok]
+    if token_major:
+        return P.T.copy()
+    M0 = M if M0 is None else M0
+    B = Ntok // L
+    cm = P.reshape(M, B, L).transpose(1, 0, 2)  # [B, M, L]
+    return cm[:, :M0].copy(), (cm[:, M0:].copy() if M0 < M else None)
