@@ -244,6 +244,37 @@ SFM_API sfm_status sfm_selective_scan_fold_bwd(const sfm_scan_args* args, const 
                                        void* workspace, size_t workspace_bytes,
                                        sfm_stream_t stream);
 
+/* Arguments of the per-token projection GEMM.  `size` must be sizeof(sfm_proj_args). */
+typedef struct {
+  uint32_t size;
+  const void* W;     /* [M, K] bf16, K contiguous (the nn.Linear weight layout)            */
+  const void* X;     /* [Ntok, K] bf16, K contiguous: one row of K features per token      */
+  void* out0;        /* channel-major: rows [0, M0) as [B, M0, L]; token-major: [Ntok, M]  */
+  void* out1;        /* channel-major: rows [M0, M) as [B, M - M0, L]; NULL if M0 == M     */
+  int M, K, Ntok;    /* Ntok = B * L tokens, sample-major                                   */
+  int M0;            /* rows written to out0 (channel-major); must equal M if token-major   */
+  int L;             /* tokens per sample                                                   */
+  int token_major;   /* 0: channel-major outputs (the scan's layout), 1: token-major out0   */
+  sfm_dtype out_dtype; /* BF16 or F32                                                       */
+  int tile_n;        /* output channels per CTA tile: 0 = automatic, 128 or 256             */
+} sfm_proj_args;
+
+/*
+ * The dense per-token maps around the scan, on the tensor cores:
+ *   P[m, n] = sum_k W[m, k] * X[n, k]      (fp32 accumulation, rounded once to out_dtype)
+ * written either channel-major -- P[m, b*L + t] at out[b, m, t], the scan's [B, rows, L]
+ * layout, so the input projection's x and z (M0 = D, M = 2D) and the state projection's
+ * B and C land where sfm_selective_scan_fold reads them -- or token-major [Ntok, M] (the
+ * low-rank step-size features that the next map reads as its X).
+ * The maps themselves are the Mamba block's input, state and step-size projections; the
+ * pages cite Mamba and MambaVision as the block's background (sungsoo.github.io, Sources
+ * and Evidence Notes, items 4 and 5) and do not spell them out.
+ * Requirements: K a multiple of 8 (16-byte row pitch), 16-byte aligned pointers, Ntok a
+ * multiple of L.  Rows or tokens past the ends are never written.  One launch.  A wait
+ * that gives up sets SFM_ERR_TIMEOUT in the device error word and skips the stores.
+ */
+SFM_API sfm_status sfm_proj_gemm(const sfm_proj_args* args, sfm_stream_t stream);
+
 /*
  * The scan backward without any allocation by the caller or the library.
  *
@@ -332,8 +363,8 @@ SFM_API sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* o
 
 /*
  * Reads (and, if clear != 0, resets) the device-side error word that kernels set when
- * a bounded wait gives up (SFM_ERR_TIMEOUT) or ragged offsets are invalid
- * (SFM_ERR_INVALID_ARG).  Synchronises `stream` first.  *code = SFM_OK when clean.
+ * a bounded wait gives up (SFM_ERR_TIMEOUT, forward or projection kernels) or ragged
+ * offsets are invalid (SFM_ERR_INVALID_ARG).  Synchronises `stream` first.  *code = SFM_OK when clean.
  */
 SFM_API sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code);
 

@@ -17,7 +17,7 @@ from ._abi import SFM_BF16, SFM_F32, SfmError
 __all__ = [
     "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d", "sfm_selective_scan_fold", "sfm_selective_scan_fold_varlen",
     "sfm_selective_scan_fold_bwd", "sfm_selective_scan_fold_bwd_noalloc", "sfm_mixer_bwd", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
-    "SfmError", "library_path",
+    "sfm_proj_gemm", "SfmError", "library_path",
 ]
 
 _DT = {torch.float32: SFM_F32, torch.bfloat16: SFM_BF16}
@@ -217,6 +217,54 @@ def sfm_selective_scan_fold_varlen(x, dt, Bm, Cm, A, cu_seqlens, *, z=None, Dski
     _abi.check(_abi.lib().sfm_selective_scan_fold_varlen(ctypes.byref(a), ctypes.c_void_p(cu_seqlens.data_ptr()),
                                                          _stream(stream)), "sfm_selective_scan_fold_varlen")
     return y
+
+
+def _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n):
+    _dev(W, "W", torch.bfloat16)
+    _dev(X, "X", torch.bfloat16)
+    if W.dim() != 2 or X.dim() != 2 or W.shape[1] != X.shape[1]:
+        raise ValueError("W must be [M, K] and X [Ntok, K], got %s and %s" % (tuple(W.shape), tuple(X.shape)))
+    M, K = W.shape
+    Ntok = X.shape[0]
+    if L < 1 or Ntok % L:
+        raise ValueError("Ntok = %d is not a multiple of L = %d" % (Ntok, L))
+    B = Ntok // L
+    M0 = M if (M0 is None or token_major) else int(M0)
+    od = torch.bfloat16 if out_dtype is None else out_dtype
+    if token_major:
+        if out0 is None:
+            out0 = torch.empty(Ntok, M, dtype=od, device=X.device)
+        _dev(out0, "out0", od, (Ntok, M))
+        out1 = None
+    else:
+        if out0 is None:
+            out0 = torch.empty(B, M0, L, dtype=od, device=X.device)
+        _dev(out0, "out0", od, (B, M0, L))
+        if M0 < M:
+            if out1 is None:
+                out1 = torch.empty(B, M - M0, L, dtype=od, device=X.device)
+            _dev(out1, "out1", od, (B, M - M0, L))
+        else:
+            out1 = None
+    a = _abi.ProjArgs()
+    a.size = ctypes.sizeof(_abi.ProjArgs)
+    a.W, a.X = W.data_ptr(), X.data_ptr()
+    a.out0 = out0.data_ptr()
+    a.out1 = out1.data_ptr() if out1 is not None else None
+    a.M, a.K, a.Ntok, a.M0, a.L = M, K, Ntok, M0, int(L)
+    a.token_major, a.out_dtype, a.tile_n = int(bool(token_major)), _code(od), int(tile_n)
+    return a, out0, out1
+
+
+def sfm_proj_gemm(W, X, L, *, M0=None, token_major=False, out_dtype=None, out0=None, out1=None, tile_n=0,
+                  stream=None):
+    """P[m, n] = sum_k W[m, k] X[n, k] on the tensor cores (bf16 in, fp32 accumulation).
+    W: [M, K] bf16; X: [Ntok, K] bf16 (tokens sample-major, L per sample).  Channel-major
+    (default): returns (out0 [B, M0, L], out1 [B, M-M0, L] or None); token-major: returns
+    (out0 [Ntok, M], None)."""
+    a, out0, out1 = _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n)
+    _abi.check(_abi.lib().sfm_proj_gemm(ctypes.byref(a), _stream(stream)), "sfm_proj_gemm")
+    return out0, out1
 
 
 def sfm_selective_scan_fold_bwd(u, dt, Bm, Cm, A, dout, *, z=None, Dskip=None, dt_bias=None, B1=0,

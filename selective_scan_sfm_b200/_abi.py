@@ -19,7 +19,7 @@ ENTRY_POINTS = (
     "sfm_status_string", "sfm_abi_version", "sfm_last_cuda_error", "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d",
     "sfm_selective_scan_fold", "sfm_scan_bwd_workspace_size", "sfm_selective_scan_fold_bwd",
     "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error", "sfm_selective_scan_fold_bwd_noalloc",
-    "sfm_mixer_bwd_workspace_size", "sfm_mixer_bwd", "sfm_selective_scan_fold_varlen",
+    "sfm_mixer_bwd_workspace_size", "sfm_mixer_bwd", "sfm_selective_scan_fold_varlen", "sfm_proj_gemm",
 )
 
 #: Size of the workspace built into the library for sfm_selective_scan_fold_bwd_noalloc.
@@ -42,6 +42,16 @@ class ScanArgs(ctypes.Structure):
         ("dt_softplus", _i), ("aux_init", _i), ("swap_out", _i),
         ("in_dtype", _i), ("out_dtype", _i),
         ("lanes", _i), ("d_tile", _i), ("chunk", _i), ("exp2_split", _i), ("chans_per_thread", _i),
+    ]
+
+
+class ProjArgs(ctypes.Structure):
+    """Mirror of sfm_proj_args."""
+    _fields_ = [
+        ("size", ctypes.c_uint32),
+        ("W", _vp), ("X", _vp), ("out0", _vp), ("out1", _vp),
+        ("M", _i), ("K", _i), ("Ntok", _i), ("M0", _i), ("L", _i),
+        ("token_major", _i), ("out_dtype", _i), ("tile_n", _i),
     ]
 
 

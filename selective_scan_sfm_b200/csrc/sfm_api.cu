@@ -526,6 +526,44 @@ sfm_status sfm_selective_scan_fold_varlen(const sfm_scan_args* a, const int* cu_
   return cuda_status(launch_fwd(p, a->in_dtype, a->out_dtype, NP, stream));
 }
 
+sfm_status sfm_proj_gemm(const sfm_proj_args* a, sfm_stream_t stream) {
+  if (!a || a->size != sizeof(sfm_proj_args) || !a->W || !a->X || !a->out0) return SFM_ERR_INVALID_ARG;
+  if (a->M < 1 || a->K < 1 || a->Ntok < 1 || a->L < 1 || a->Ntok % a->L != 0) return SFM_ERR_INVALID_ARG;
+  if ((a->token_major & ~1) || !dtype_ok(a->out_dtype)) return SFM_ERR_INVALID_ARG;
+  if (a->token_major ? (a->M0 != a->M || a->out1) : (a->M0 < 1 || a->M0 > a->M || ((a->M0 < a->M) != !!a->out1)))
+    return SFM_ERR_INVALID_ARG;
+  if (a->tile_n != 0 && a->tile_n != 128 && a->tile_n != 256) return SFM_ERR_UNSUPPORTED;
+  if (a->K % 8 != 0) return SFM_ERR_UNSUPPORTED;  // TMA: the row pitch of W and X is a multiple of 16 bytes
+  const void* ptrs[] = {a->W, a->X, a->out0, a->out1};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return SFM_ERR_MISALIGNED;
+  const long long os = esize_of(a->out_dtype);
+  const long long wb = (long long)a->M * a->K * 2, xb = (long long)a->Ntok * a->K * 2;
+  const long long o0 = (long long)a->Ntok * (a->token_major ? a->M : a->M0) * os;
+  const long long o1 = (long long)a->Ntok * (a->M - a->M0) * os;
+  if (overlaps(a->out0, o0, a->W, wb) || overlaps(a->out0, o0, a->X, xb) || overlaps(a->out1, o1, a->W, wb) ||
+      overlaps(a->out1, o1, a->X, xb) || overlaps(a->out0, o0, a->out1, o1))
+    return SFM_ERR_INVALID_ARG;
+  ProjParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.W = a->W;
+  p.X = a->X;
+  p.out0 = a->out0;
+  p.out1 = a->out1;
+  p.M = a->M;
+  p.K = a->K;
+  p.Ntok = a->Ntok;
+  p.M0 = a->M0;
+  p.L = a->L;
+  p.token_major = a->token_major;
+  p.out_f32 = a->out_dtype == SFM_F32;
+  // 128 channels per tile for the short K of the projections (more, smaller CTAs: their
+  // epilogue stores overlap the others' loads), 256 when K is long and the MMAs dominate
+  p.bn = a->tile_n ? a->tile_n : (a->K > 640 ? 256 : 128);
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_proj(p, stream));
+}
+
 sfm_status sfm_scan_bwd_workspace_size(const sfm_scan_args* a, size_t* bytes) {
   if (!bytes) return SFM_ERR_INVALID_ARG;
   const sfm_status st = validate_bwd_args(a);
@@ -611,10 +649,12 @@ sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* a, const sfm
 
 sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code) {
   if (!code) return SFM_ERR_INVALID_ARG;
-  unsigned v = 0;
-  const sfm_status st = cuda_status(read_device_error(stream, clear, &v));
+  unsigned v = 0, w = 0;
+  sfm_status st = cuda_status(read_device_error(stream, clear, &v));
   if (st != SFM_OK) return st;
-  *code = (int)v;
+  st = cuda_status(read_proj_error(clear, &w));  // the projection kernels' word
+  if (st != SFM_OK) return st;
+  *code = (int)(v ? v : w);
   return SFM_OK;
 }
 

@@ -185,4 +185,52 @@ __device__ __forceinline__ void store_row(T* base, long long e0, const char* src
 
 __device__ __forceinline__ int span_head(long long e0, int esize) { return (int)((e0 * esize) & 15); }
 
+
+// ------------------------------------------------------------------ mbarriers with bounded waits
+
+constexpr unsigned long long kWaitNs = 2000000000ull;  // every wait on an mbarrier gives up after 2 s
+
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Polls the barrier until the phase with `parity` completes or kWaitNs elapse.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kWaitNs) return false;
+  return true;
+}
+
+// The same bounded wait for threads off the critical path (a whole CTA waiting for its
+// accumulator): they sleep between polls so co-resident CTAs keep the issue slots.
+__device__ __forceinline__ bool mbar_wait_bounded_sleepy(uint64_t* bar, unsigned parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    __nanosleep(256);
+    if (global_ns() - t0 > kWaitNs) return false;
+  }
+  return true;
+}
+
 }  // namespace sfm

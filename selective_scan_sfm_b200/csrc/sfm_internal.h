@@ -56,6 +56,18 @@ constexpr int kModeWhole = 1;
 constexpr int kModeLanes = 2;  // P lanes per channel split the tokens (warp-shuffle scan)
 constexpr int kLaneTokens = 16;  // tokens per lane per chunk in kModeLanes
 
+// The per-token projection GEMM: P[m, n] = sum_k W[m, k] * X[n, k].
+struct ProjParams {
+  const void* W;    // [M, K] bf16
+  const void* X;    // [Ntok, K] bf16
+  void* out0;       // channel-major [B, M0, L] (rows [0, M0)) or token-major [Ntok, M]
+  void* out1;       // channel-major [B, M - M0, L] (rows [M0, M)), or NULL
+  int M, K, Ntok, M0, L;
+  int token_major;  // 1: out0 is [Ntok, M]
+  int out_f32;      // 1: fp32 outputs, else bf16
+  int bn;           // output channels per CTA tile: 128 or 256
+};
+
 struct BwdParams {
   const void* u;
   const void* dt;
@@ -89,6 +101,8 @@ int fwd_max_smem();
 int fwd_x_row(int chunk, int K, int esize);
 int fwd_io_row(int chunk, int esize);
 int fwd_y_row(int chunk, int esize);
+cudaError_t launch_proj(const ProjParams& p, cudaStream_t s);
+cudaError_t read_proj_error(int clear, unsigned* value);
 cudaError_t read_device_error(cudaStream_t s, int clear, unsigned* value);
 
 cudaError_t launch_bwd(const BwdParams& p, sfm_dtype in_dtype, sfm_dtype dout_dtype, cudaStream_t s);
