@@ -118,6 +118,15 @@ SFM_API sfm_status sfm_fold_conv1d(const void* x, const float* w, const float* b
                            int B, int D, int L, int K, int pad_left, int B2, int silu,
                            sfm_dtype dtype, sfm_stream_t stream);
 
+/*
+ * The conv of sfm_fold_conv1d (same arguments and zero padding per sample) written
+ * token-major: u [B*L, D] (row b*L + t holds the D channels of token t of sample b), the
+ * layout the state projection (sfm_proj_gemm) reads as X.  x [B,D,L] and u must not
+ * overlap.  Same sources as sfm_fold_conv1d.
+ */
+SFM_API sfm_status sfm_conv1d_tokens(const void* x, const float* w, const float* bias, void* u, int B, int D,
+                                     int L, int K, int pad_left, int silu, sfm_dtype dtype, sfm_stream_t stream);
+
 /* Arguments of the fused folded scan.  `size` must be sizeof(sfm_scan_args). */
 typedef struct {
   uint32_t size;

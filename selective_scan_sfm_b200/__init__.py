@@ -17,7 +17,7 @@ from ._abi import SFM_BF16, SFM_F32, SfmError
 __all__ = [
     "sfm_aux_init", "sfm_aux_swap", "sfm_fold_conv1d", "sfm_selective_scan_fold", "sfm_selective_scan_fold_varlen",
     "sfm_selective_scan_fold_bwd", "sfm_selective_scan_fold_bwd_noalloc", "sfm_mixer_bwd", "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error",
-    "sfm_proj_gemm", "SfmError", "library_path",
+    "sfm_proj_gemm", "sfm_conv1d_tokens", "SfmError", "library_path",
 ]
 
 _DT = {torch.float32: SFM_F32, torch.bfloat16: SFM_BF16}
@@ -217,6 +217,22 @@ def sfm_selective_scan_fold_varlen(x, dt, Bm, Cm, A, cu_seqlens, *, z=None, Dski
     _abi.check(_abi.lib().sfm_selective_scan_fold_varlen(ctypes.byref(a), ctypes.c_void_p(cu_seqlens.data_ptr()),
                                                          _stream(stream)), "sfm_selective_scan_fold_varlen")
     return y
+
+
+def sfm_conv1d_tokens(x, w, bias=None, *, pad_left=None, silu=True, u=None, stream=None):
+    """Boundary-safe depthwise conv (+SiLU) of x [B,D,L], written token-major u [B*L, D]."""
+    _dev(x, "x")
+    B, D, L = x.shape
+    K = w.shape[1]
+    _dev(w, "w", torch.float32, (D, K))
+    _dev(bias, "bias", torch.float32, (D,), optional=True)
+    if u is None:
+        u = torch.empty(B * L, D, dtype=x.dtype, device=x.device)
+    _dev(u, "u", x.dtype, (B * L, D))
+    pl = (K - 1) // 2 if pad_left is None else int(pad_left)
+    _abi.check(_abi.lib().sfm_conv1d_tokens(_ptr(x), _ptr(w), _ptr(bias), _ptr(u), B, D, L, K, pl, int(bool(silu)),
+                                            _code(x.dtype), _stream(stream)), "sfm_conv1d_tokens")
+    return u
 
 
 def _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n):

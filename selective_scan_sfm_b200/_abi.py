@@ -20,6 +20,7 @@ ENTRY_POINTS = (
     "sfm_selective_scan_fold", "sfm_scan_bwd_workspace_size", "sfm_selective_scan_fold_bwd",
     "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error", "sfm_selective_scan_fold_bwd_noalloc",
     "sfm_mixer_bwd_workspace_size", "sfm_mixer_bwd", "sfm_selective_scan_fold_varlen", "sfm_proj_gemm",
+    "sfm_conv1d_tokens",
 )
 
 #: Size of the workspace built into the library for sfm_selective_scan_fold_bwd_noalloc.

@@ -327,6 +327,18 @@ sfm_status sfm_fold_conv1d(const void* x, const float* w, const float* bias, voi
   return cuda_status(launch_conv1d(x, w, bias, u, B, D, L, K, pad_left, silu, dtype, stream));
 }
 
+sfm_status sfm_conv1d_tokens(const void* x, const float* w, const float* bias, void* u, int B, int D, int L, int K,
+                             int pad_left, int silu, sfm_dtype dtype, sfm_stream_t stream) {
+  if (!x || !w || !u || B < 1 || D < 1 || L < 1 || !dtype_ok(dtype)) return SFM_ERR_INVALID_ARG;
+  if (K < 1 || K > SFM_MAX_K || pad_left < 0 || pad_left >= K || (silu & ~1)) return SFM_ERR_INVALID_ARG;
+  if (L > SFM_MAX_L || B > 65535) return SFM_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(u)) return SFM_ERR_MISALIGNED;
+  const long long bytes = (long long)B * D * L * esize_of(dtype);
+  if (overlaps(x, bytes, u, bytes)) return SFM_ERR_INVALID_ARG;
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_conv1d_tokens(x, w, bias, u, B, D, L, K, pad_left, silu, dtype, stream));
+}
+
 sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* out) {
   if (!out || B < 1 || T < 1 || D < 1 || N < 1) return SFM_ERR_INVALID_ARG;
   *out = choose(B, T, D, N);

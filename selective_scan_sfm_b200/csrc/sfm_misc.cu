@@ -75,7 +75,48 @@ __global__ void conv1d_kernel(const T* __restrict__ x, const float* __restrict__
   }
 }
 
+// The same conv written token-major, u[b*L + t, d]: the layout the state projection reads
+// (one row of D features per token).  A CTA takes 32 tokens x 64 channels of one sample:
+// the x rows it needs (with the taps' halo, zero outside the sample) are staged in shared
+// memory by coalesced row reads, and each token's 64 channels leave as one contiguous run.
+template <typename T>
+__global__ void __launch_bounds__(256) conv1d_tokens_kernel(const T* __restrict__ x, const float* __restrict__ w,
+                                                            const float* __restrict__ bias, T* __restrict__ u,
+                                                            int D, int L, int K, int pad_left, int silu_on) {
+  constexpr int TT = 32, DT = 64, HALO = SFM_MAX_K - 1, ROW = TT + HALO + 1;  // odd row stride: no bank conflicts
+  __shared__ float xs[DT][ROW];
+  const int t0 = blockIdx.x * TT, d0 = blockIdx.y * DT, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  for (int e = tid; e < DT * (TT + HALO); e += blockDim.x) {
+    const int c = e / (TT + HALO), i = e % (TT + HALO);
+    const int d = d0 + c, s = t0 - pad_left + i;
+    xs[c][i] = (d < D && s >= 0 && s < L) ? to_f(x[((size_t)b * D + d) * L + s]) : 0.0f;
+  }
+  __syncthreads();
+  for (int e = tid; e < TT * DT; e += blockDim.x) {
+    const int i = e / DT, c = e % DT;  // channel fastest: the stores of a token are contiguous
+    const int t = t0 + i, d = d0 + c;
+    if (t >= L || d >= D) continue;
+    float acc = bias ? bias[d] : 0.0f;
+    for (int k = 0; k < K; ++k) acc = fmaf(w[(size_t)d * K + k], xs[c][i + k], acc);
+    u[((size_t)b * L + t) * D + d] = from_f<T>(silu_on ? silu(acc) : acc);
+  }
+}
+
 static unsigned blocks_for(long long items, int per_block) { return (unsigned)((items + per_block - 1) / per_block); }
+
+cudaError_t launch_conv1d_tokens(const void* x, const float* w, const float* bias, void* u, int B, int D, int L,
+                                 int K, int pad_left, int silu_on, sfm_dtype dtype, cudaStream_t s) {
+  dim3 grid((L + 31) / 32, (D + 63) / 64, B);
+  if (dtype == SFM_F32)
+    conv1d_tokens_kernel<float><<<grid, 256, 0, s>>>(static_cast<const float*>(x), w, bias, static_cast<float*>(u),
+                                                     D, L, K, pad_left, silu_on);
+  else
+    conv1d_tokens_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), w, bias,
+                                                             static_cast<__nv_bfloat16*>(u), D, L, K, pad_left,
+                                                             silu_on);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_aux_init(const void* x, void* xa, int B, int D, int T, int esize, cudaStream_t s) {
   const long long rows = (long long)B * D;

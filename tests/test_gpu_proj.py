@@ -89,3 +89,69 @@ def test_validation():
     W, X = draw(128, 64, 64, seed=3)
     with pytest.raises(ValueError):
         sfm_proj_gemm(W.cuda(), X.cuda(), 48)  # 64 tokens are not whole samples of 48
+
+
+# ------------------------------------------------------------------ the path around the scan
+
+from selective_scan_sfm_b200 import sfm_conv1d_tokens, sfm_selective_scan_fold  # noqa: E402
+
+from parity import TOL, bf16_round, rel_err  # noqa: E402
+
+
+@pytest.mark.parametrize("dt,pad_left", [(torch.float32, 1), (torch.bfloat16, 3), (torch.bfloat16, 0)])
+def test_conv1d_tokens(dt, pad_left):
+    g = torch.Generator().manual_seed(70 + pad_left)
+    B, D, L = 3, 100, 77
+    x = torch.randn(B, D, L, generator=g).to(dt)
+    w = torch.rand(D, 4, generator=g) - 0.5
+    bias = torch.rand(D, generator=g) - 0.5
+    u = sfm_conv1d_tokens(x.cuda(), w.cuda(), bias.cuda(), pad_left=pad_left)
+    ref = oracle.conv1d(x.double().numpy(), w.double().numpy(), bias.double().numpy(), pad_left=pad_left, silu=True)
+    ref = ref.transpose(0, 2, 1).reshape(B * L, D)
+    got = u.double().cpu().numpy()
+    if dt == torch.float32:
+        assert rel_err(got, ref) <= TOL["f32"]
+    else:
+        assert rel_err(got, bf16_round(ref)) <= 2.0 ** -7  # bf16 RN on both sides, fp32 vs fp64 sums
+
+
+def test_projections_feed_the_scan():
+    """tokens -> in_proj (x, z) -> conv (token-major u) -> x_proj (dt_low, B, C) -> dt_proj
+    (dt) -> the fused scan, all on the GPU, against the same chain in the oracle (fp64,
+    rounded to bf16 at the same stage boundaries, on its own values)."""
+    g = torch.Generator().manual_seed(77)
+    B, L, C, D, N, R = 4, 51, 160, 320, 16, 24
+    bf = torch.bfloat16
+    tok = torch.randn(B * L, C, generator=g).to(bf)
+    W_in = (torch.randn(2 * D, C, generator=g) / C ** 0.5).to(bf)
+    W_x = (torch.randn(R + 2 * N, D, generator=g) / D ** 0.5).to(bf)
+    W_dt = (0.5 * torch.randn(D, R, generator=g) / R ** 0.5).to(bf)
+    conv_w = torch.rand(D, 4, generator=g) - 0.5
+    conv_b = torch.rand(D, generator=g) - 0.5
+    A = -torch.exp(torch.randn(D, N, generator=g))
+    Dskip = torch.randn(D, generator=g)
+    dt_bias = torch.log(torch.expm1(1e-3 + torch.rand(D, generator=g, dtype=torch.float64) * (1e-1 - 1e-3))).float()
+    c = lambda t: t.cuda()
+    x, z = sfm_proj_gemm(c(W_in), c(tok), L, M0=D)
+    u_tok = sfm_conv1d_tokens(x, c(conv_w), c(conv_b))
+    dt_low, _ = sfm_proj_gemm(c(W_x[:R].contiguous()), u_tok, L, token_major=True)
+    Bm, Cm = sfm_proj_gemm(c(W_x[R:].contiguous()), u_tok, L, M0=N)
+    dt, _ = sfm_proj_gemm(c(W_dt), dt_low, L)
+    y = sfm_selective_scan_fold(x, dt, Bm, Cm, c(A), z=z, Dskip=c(Dskip), dt_bias=c(dt_bias), conv_w=c(conv_w),
+                                conv_b=c(conv_b))
+    torch.cuda.synchronize()
+    assert sfm_get_device_error(clear=True) == 0
+
+    f = lambda t: t.double().numpy()
+    r16 = bf16_round
+    xr, zr = oracle.proj(f(W_in), f(tok), L, M0=D)
+    xr, zr = r16(xr), r16(zr)
+    ur = r16(oracle.conv1d(xr, f(conv_w), f(conv_b), silu=True).transpose(0, 2, 1).reshape(B * L, D))
+    dlr = r16(oracle.proj(f(W_x[:R]), ur, L, token_major=True))
+    br, cr = oracle.proj(f(W_x[R:]), ur, L, M0=N)
+    br, cr = r16(br), r16(cr)
+    dtr, _ = oracle.proj(f(W_dt), dlr, L)
+    dtr = r16(dtr)
+    yr = oracle.mixer_layer(xr, dtr, zr, br, cr, f(A), f(Dskip), f(dt_bias), f(conv_w), f(conv_b))
+    e = rel_err(y.double().cpu().numpy(), yr)
+    assert e <= TOL["bf16"], e
