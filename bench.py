@@ -108,12 +108,15 @@ def mufu_only_peak_elems(N, K, sm_mhz, sms=SMS):
     return sms * sm_mhz * 1e6 / max(E / MUFU_PER_CLK_SM, F / FP32_PER_CLK_SM)
 
 
+# the sources that decide the benchmark kernel and its launch shape
+FWD_SOURCES = ("sfm_fwd.cu", "sfm_device.cuh", "sfm_internal.h", "sfm_api.cu", "sfm_lut.inc")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "selective_scan_sfm_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h", ".inc")):
-            h.update(open(os.path.join(csrc, f), "rb").read())
+    for f in FWD_SOURCES:
+        h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -441,6 +444,47 @@ def measure_ragged(steps, warmup, world, rank, device, seed_base=0, workload="ra
                 padded_total_ms=ptotal_ms, padded_launch_ms=plaunch_ms, padded_elements=S * D * (Tmax + 2))
 
 
+def measure_proj(steps, warmup, world, device, workload="stage4_t49", seed=0):
+    """The projections around the scan at a workload's shape, each a tcgen05 GEMM timed on
+    its own: in_proj (tokens [B*L, D/2] -> x, z [B,D,L]), x_proj (u [B*L, D] -> dt_low
+    token-major [B*L, R], B and C [B,N,L]) and dt_proj (dt_low -> dt [B,D,L]), with
+    d_model = D/2 and R = ceil(D/16) (the Mamba defaults; the pages fix neither)."""
+    import torch
+    from selective_scan_sfm_b200 import _abi, _proj_args, synth
+
+    w = synth.WORKLOADS[workload]
+    B, D, L, N = w["B"], w["D"], w["T"] + 2, w["N"]
+    C, R = D // 2, -(-D // 16)
+    R = -(-R // 8) * 8  # a multiple of 8 (16-byte rows for the tensor maps)
+    Ntok = B * L
+    g = torch.Generator().manual_seed(seed)
+    bf = torch.bfloat16
+    mk = lambda *sh, scale=1.0: (scale * torch.randn(*sh, generator=g)).to(bf).to(device)
+    tok, u = mk(Ntok, C), mk(Ntok, D)
+    W_in, W_x, W_dt = mk(2 * D, C, scale=C ** -0.5), mk(R + 2 * N, D, scale=D ** -0.5), mk(D, R, scale=R ** -0.5)
+    dt_low = mk(Ntok, R)
+    gemms = {
+        "in_proj": (_proj_args(W_in, tok, L, D, False, bf, None, None, 0)[0], 2.0 * Ntok * C * 2 * D),
+        "x_proj_bc": (_proj_args(W_x[R:].contiguous(), u, L, N, False, bf, None, None, 0)[0], 2.0 * Ntok * D * 2 * N),
+        "x_proj_dt": (_proj_args(W_x[:R].contiguous(), u, L, None, True, bf, None, None, 0)[0], 2.0 * Ntok * D * R),
+        "dt_proj": (_proj_args(W_dt, dt_low, L, D, False, bf, None, None, 0)[0], 2.0 * Ntok * R * D),
+    }
+    keep = (tok, u, W_in, W_x, W_dt, dt_low)  # noqa: F841  (the args point into these)
+    lib = _abi.lib()
+    stream = torch.cuda.current_stream(device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    out = {}
+    for name, (a, flops) in gemms.items():
+        def launch(i, a=a):
+            rc = lib.sfm_proj_gemm(ctypes.byref(a), sp)
+            if rc != 0:
+                raise RuntimeError(_abi.status_string(rc))
+        _, ms = _time_launches(launch, 1, steps, warmup, world, device, stream)
+        out[name] = dict(ms=ms, flops=flops)
+    out["shape"] = dict(B=B, L=L, d_model=C, D=D, N=N, R=R)
+    return out
+
+
 def max_over_ranks(v, world, device):
     if world == 1:
         return v
@@ -526,6 +570,13 @@ def main(argv=None):
                                            "padded to the longest (%d of %d elements useful)"
                                            % (rr["elements"], rr["padded_elements"])}}
 
+    proj = {}
+    if not args.no_extra:
+        pr = measure_proj(args.steps, args.warmup, world, device)
+        proj = {k: v for k, v in pr.items()}
+        for k in ("in_proj", "x_proj_bc", "x_proj_dt", "dt_proj"):
+            proj[k]["ms"] = max_over_ranks(proj[k]["ms"], world, device)
+
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -588,6 +639,16 @@ def main(argv=None):
         line["t196"] = extra
     if ragged:
         line["ragged"] = ragged
+    if proj:
+        bf_peak = float(peaks.get("bf16_tflops", 1590.0)) if peaks else 1590.0
+        bf_sus = float(peaks.get("bf16_tflops_sustained", 1400.0)) if peaks else 1400.0
+        pj = {"workload": "stage4_t49 projections (tcgen05 GEMMs, bf16 in, fp32 accumulate, bf16 out)",
+              "shape": proj["shape"], "peak_tflops": bf_peak, "peak_tflops_sustained": bf_sus,
+              "peak_source": "measured" if peaks else "fallback"}
+        for k in ("in_proj", "x_proj_bc", "x_proj_dt", "dt_proj"):
+            tf = proj[k]["flops"] / (proj[k]["ms"] * 1e-3) / 1e12
+            pj[k] = {"ms": proj[k]["ms"], "tflops": tf, "frac": tf / bf_peak}
+        line["proj"] = pj
     if cpu:
         line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
