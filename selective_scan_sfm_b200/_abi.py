@@ -108,6 +108,9 @@ def lib():
         L.sfm_choose_variant.argtypes = [_i, _i, _i, _i, ctypes.POINTER(Variant)]
         L.sfm_get_device_error.argtypes = [_vp, _i, ctypes.POINTER(_i)]
         L.sfm_selective_scan_fold_bwd_noalloc.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ScanGrads), _vp]
+        L.sfm_selective_scan_fold_varlen.argtypes = [ctypes.POINTER(ScanArgs), _vp, _vp]
+        L.sfm_proj_gemm.argtypes = [ctypes.POINTER(ProjArgs), _vp]
+        L.sfm_conv1d_tokens.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
         L.sfm_mixer_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ctypes.c_size_t)]
         L.sfm_mixer_bwd.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(MixerGrads), _vp, ctypes.c_size_t, _vp]
         for name in ENTRY_POINTS:

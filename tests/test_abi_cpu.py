@@ -200,3 +200,74 @@ def test_mixer_backward_validation(L, inject):
     assert call(good_args(), g) == _abi.SFM_ERR_INVALID_ARG          # conv given, no dconv_w
     g.dconv_w = FAKE + (1 << 24)                                      # aliases dt
     assert call(good_args(), g) == _abi.SFM_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------------------ ragged folding, projections
+
+def varlen_args(**kw):
+    # 5 samples packed into 60 positions (>= 3 per sample with aux tokens)
+    return good_args(**dict(dict(B=5, L=60, B1=0, reset_period=0), **kw))
+
+
+CU = FAKE + (11 << 24)
+
+
+def test_varlen_validation(L, inject):
+    v = L.sfm_selective_scan_fold_varlen
+    assert v(ctypes.byref(varlen_args()), CU, None) == _abi.SFM_ERR_CUDA
+    assert v(ctypes.byref(varlen_args(L=20000)), CU, None) == _abi.SFM_ERR_CUDA  # no per-sample cap on the total
+    assert v(ctypes.byref(varlen_args()), None, None) == _abi.SFM_ERR_INVALID_ARG
+    assert v(ctypes.byref(varlen_args()), CU + 2, None) == _abi.SFM_ERR_MISALIGNED
+    assert v(ctypes.byref(varlen_args(reset_period=60)), CU, None) == _abi.SFM_ERR_UNSUPPORTED
+    assert v(ctypes.byref(varlen_args(lanes=2)), CU, None) == _abi.SFM_ERR_UNSUPPORTED
+    assert v(ctypes.byref(varlen_args(N=17)), CU, None) == _abi.SFM_ERR_UNSUPPORTED
+    assert v(ctypes.byref(varlen_args(L=14)), CU, None) == _abi.SFM_ERR_INVALID_ARG   # < 3 tokens per sample
+    assert v(ctypes.byref(varlen_args(B1=2)), CU, None) == _abi.SFM_ERR_INVALID_ARG   # does not divide 5
+    assert v(ctypes.byref(varlen_args(y=CU)), CU, None) == _abi.SFM_ERR_INVALID_ARG  # output aliases the offsets
+
+
+def proj_args(**kw):
+    a = _abi.ProjArgs()
+    a.size = ctypes.sizeof(_abi.ProjArgs)
+    a.W, a.X, a.out0, a.out1 = FAKE, FAKE + (1 << 24), FAKE + (2 << 24), FAKE + (3 << 24)
+    a.M, a.K, a.Ntok, a.M0, a.L = 256, 64, 4 * 51, 128, 51
+    a.token_major, a.out_dtype, a.tile_n = 0, _abi.SFM_BF16, 0
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("size", 8, _abi.SFM_ERR_INVALID_ARG),
+    ("W", None, _abi.SFM_ERR_INVALID_ARG),
+    ("out0", None, _abi.SFM_ERR_INVALID_ARG),
+    ("K", 60, _abi.SFM_ERR_UNSUPPORTED),            # rows not a multiple of 16 bytes
+    ("Ntok", 4 * 51 + 1, _abi.SFM_ERR_INVALID_ARG),  # not whole samples
+    ("M0", 300, _abi.SFM_ERR_INVALID_ARG),
+    ("out1", None, _abi.SFM_ERR_INVALID_ARG),       # M0 < M needs the second output
+    ("token_major", 1, _abi.SFM_ERR_INVALID_ARG),   # token-major writes one output of all M rows
+    ("tile_n", 64, _abi.SFM_ERR_UNSUPPORTED),
+    ("out_dtype", 5, _abi.SFM_ERR_INVALID_ARG),
+    ("X", FAKE + (1 << 24) + 8, _abi.SFM_ERR_MISALIGNED),
+    ("out0", FAKE + (1 << 24), _abi.SFM_ERR_INVALID_ARG),  # output aliases X
+])
+def test_proj_validation(L, inject, field, value, code):
+    assert L.sfm_proj_gemm(ctypes.byref(proj_args(**{field: value})), None) == code
+
+
+def test_proj_valid_args_reach_the_launch_path(L, inject):
+    assert L.sfm_proj_gemm(ctypes.byref(proj_args()), None) == _abi.SFM_ERR_CUDA
+    assert L.sfm_proj_gemm(ctypes.byref(proj_args(token_major=1, M0=256, out1=None)), None) == _abi.SFM_ERR_CUDA
+    assert L.sfm_proj_gemm(ctypes.byref(proj_args(M0=256, out1=None, tile_n=256, out_dtype=_abi.SFM_F32)),
+                           None) == _abi.SFM_ERR_CUDA
+
+
+def test_conv1d_tokens_validation(L, inject):
+    c = L.sfm_conv1d_tokens
+    W, U = FAKE + (1 << 24), FAKE + (2 << 24)
+    assert c(FAKE, W, None, U, 2, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_CUDA
+    assert c(FAKE, W, None, U, 0, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_INVALID_ARG
+    assert c(FAKE, W, None, U, 2, 64, 51, 4, 4, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_INVALID_ARG
+    assert c(FAKE, None, None, U, 2, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_INVALID_ARG
+    assert c(FAKE, W, None, U + 2, 2, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_MISALIGNED
+    assert c(FAKE, W, None, FAKE + 16, 2, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_INVALID_ARG
