@@ -377,6 +377,14 @@ SFM_API sfm_status sfm_choose_variant(int B, int T, int D, int N, sfm_variant* o
  */
 SFM_API sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code);
 
+/*
+ * Self-test of the bounded-wait path: launches one thread that waits on an mbarrier
+ * nothing arrives on, gives up after limit_us microseconds (1 .. 1e6), records
+ * SFM_ERR_TIMEOUT in the device error word exactly as the kernels' own waits do, and
+ * returns.  Nothing faults or hangs; read the result with sfm_get_device_error.
+ */
+SFM_API sfm_status sfm_selftest_wait_timeout(int limit_us, sfm_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -20,7 +20,7 @@ ENTRY_POINTS = (
     "sfm_selective_scan_fold", "sfm_scan_bwd_workspace_size", "sfm_selective_scan_fold_bwd",
     "sfm_choose_b1", "sfm_choose_variant", "sfm_get_device_error", "sfm_selective_scan_fold_bwd_noalloc",
     "sfm_mixer_bwd_workspace_size", "sfm_mixer_bwd", "sfm_selective_scan_fold_varlen", "sfm_proj_gemm",
-    "sfm_conv1d_tokens",
+    "sfm_conv1d_tokens", "sfm_selftest_wait_timeout",
 )
 
 #: Size of the workspace built into the library for sfm_selective_scan_fold_bwd_noalloc.
@@ -111,6 +111,7 @@ def lib():
         L.sfm_selective_scan_fold_varlen.argtypes = [ctypes.POINTER(ScanArgs), _vp, _vp]
         L.sfm_proj_gemm.argtypes = [ctypes.POINTER(ProjArgs), _vp]
         L.sfm_conv1d_tokens.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _vp]
+        L.sfm_selftest_wait_timeout.argtypes = [_i, _vp]
         L.sfm_mixer_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(ctypes.c_size_t)]
         L.sfm_mixer_bwd.argtypes = [ctypes.POINTER(ScanArgs), ctypes.POINTER(MixerGrads), _vp, ctypes.c_size_t, _vp]
         for name in ENTRY_POINTS:

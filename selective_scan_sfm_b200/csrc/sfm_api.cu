@@ -659,6 +659,12 @@ sfm_status sfm_selective_scan_fold_bwd_noalloc(const sfm_scan_args* a, const sfm
   return cuda_status(launch_bwd(p, a->in_dtype, a->out_dtype, stream));
 }
 
+sfm_status sfm_selftest_wait_timeout(int limit_us, sfm_stream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return SFM_ERR_INVALID_ARG;
+  if (fault_injected()) return SFM_ERR_CUDA;
+  return cuda_status(launch_wait_selftest(limit_us, stream));
+}
+
 sfm_status sfm_get_device_error(sfm_stream_t stream, int clear, int* code) {
   if (!code) return SFM_ERR_INVALID_ARG;
   unsigned v = 0, w = 0;

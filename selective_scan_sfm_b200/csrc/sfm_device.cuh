@@ -221,6 +221,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, unsigned parity
   return true;
 }
 
+// A bounded wait with an explicit limit in nanoseconds (the self-test of the timeout path).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, unsigned parity, unsigned long long limit_ns) {
+  const unsigned long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    __nanosleep(1000);
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+  return true;
+}
+
 // The same bounded wait for threads off the critical path (a whole CTA waiting for its
 // accumulator): they sleep between polls so co-resident CTAs keep the issue slots.
 __device__ __forceinline__ bool mbar_wait_bounded_sleepy(uint64_t* bar, unsigned parity) {

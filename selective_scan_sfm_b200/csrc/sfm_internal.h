@@ -104,6 +104,7 @@ int fwd_y_row(int chunk, int esize);
 cudaError_t launch_conv1d_tokens(const void* x, const float* w, const float* bias, void* u, int B, int D, int L,
                                  int K, int pad_left, int silu_on, sfm_dtype dtype, cudaStream_t s);
 cudaError_t launch_proj(const ProjParams& p, cudaStream_t s);
+cudaError_t launch_wait_selftest(int limit_us, cudaStream_t s);
 cudaError_t read_proj_error(int clear, unsigned* value);
 cudaError_t read_device_error(cudaStream_t s, int clear, unsigned* value);
 

@@ -333,6 +333,22 @@ cudaError_t launch_proj(const ProjParams& p, cudaStream_t s) {
   return p.out_f32 ? launch_to<float>(p, s) : launch_to<__nv_bfloat16>(p, s);
 }
 
+// Self-test of the timeout path: one thread waits on an mbarrier that nothing will ever
+// arrive on, with a limit of limit_us; when the wait gives up it records SFM_ERR_TIMEOUT
+// in the device error word, exactly as the kernels' own waits do, and returns.
+__global__ void wait_timeout_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  if (!mbar_wait_for(&bar, 0, limit_ns)) atomicExch(&g_proj_error, (unsigned)SFM_ERR_TIMEOUT);
+}
+
+cudaError_t launch_wait_selftest(int limit_us, cudaStream_t s) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, s>>>(1000ull * (unsigned long long)limit_us);
+  return cudaGetLastError();
+}
+
 cudaError_t read_proj_error(int clear, unsigned* value) {
   cudaError_t e = cudaMemcpyFromSymbol(value, g_proj_error, sizeof(unsigned));
   if (e != cudaSuccess || !clear) return e;

@@ -271,3 +271,9 @@ def test_conv1d_tokens_validation(L, inject):
     assert c(FAKE, None, None, U, 2, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_INVALID_ARG
     assert c(FAKE, W, None, U + 2, 2, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_MISALIGNED
     assert c(FAKE, W, None, FAKE + 16, 2, 64, 51, 4, 1, 1, _abi.SFM_BF16, None) == _abi.SFM_ERR_INVALID_ARG
+
+
+def test_selftest_wait_validation(L, inject):
+    assert L.sfm_selftest_wait_timeout(0, None) == _abi.SFM_ERR_INVALID_ARG
+    assert L.sfm_selftest_wait_timeout(2000000, None) == _abi.SFM_ERR_INVALID_ARG
+    assert L.sfm_selftest_wait_timeout(100, None) == _abi.SFM_ERR_CUDA  # reached the launch path
