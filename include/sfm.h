@@ -266,6 +266,8 @@ typedef struct {
   int token_major;   /* 0: channel-major outputs (the scan's layout), 1: token-major out0   */
   sfm_dtype out_dtype; /* BF16 or F32                                                       */
   int tile_n;        /* output channels per CTA tile: 0 = automatic, 128 or 256             */
+  int schedule;      /* 0 = automatic, 1 = one CTA per tile, 2 = persistent (one CTA per SM
+                        walking its tiles, the epilogue overlapping the next tile's MMAs)   */
 } sfm_proj_args;
 
 /*

@@ -235,7 +235,7 @@ def sfm_conv1d_tokens(x, w, bias=None, *, pad_left=None, silu=True, u=None, stre
     return u
 
 
-def _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n):
+def _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n, schedule=0):
     _dev(W, "W", torch.bfloat16)
     _dev(X, "X", torch.bfloat16)
     if W.dim() != 2 or X.dim() != 2 or W.shape[1] != X.shape[1]:
@@ -269,16 +269,17 @@ def _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n):
     a.out1 = out1.data_ptr() if out1 is not None else None
     a.M, a.K, a.Ntok, a.M0, a.L = M, K, Ntok, M0, int(L)
     a.token_major, a.out_dtype, a.tile_n = int(bool(token_major)), _code(od), int(tile_n)
+    a.schedule = int(schedule)
     return a, out0, out1
 
 
 def sfm_proj_gemm(W, X, L, *, M0=None, token_major=False, out_dtype=None, out0=None, out1=None, tile_n=0,
-                  stream=None):
+                  schedule=0, stream=None):
     """P[m, n] = sum_k W[m, k] X[n, k] on the tensor cores (bf16 in, fp32 accumulation).
     W: [M, K] bf16; X: [Ntok, K] bf16 (tokens sample-major, L per sample).  Channel-major
     (default): returns (out0 [B, M0, L], out1 [B, M-M0, L] or None); token-major: returns
     (out0 [Ntok, M], None)."""
-    a, out0, out1 = _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n)
+    a, out0, out1 = _proj_args(W, X, L, M0, token_major, out_dtype, out0, out1, tile_n, schedule)
     _abi.check(_abi.lib().sfm_proj_gemm(ctypes.byref(a), _stream(stream)), "sfm_proj_gemm")
     return out0, out1
 

@@ -52,7 +52,7 @@ class ProjArgs(ctypes.Structure):
         ("size", ctypes.c_uint32),
         ("W", _vp), ("X", _vp), ("out0", _vp), ("out1", _vp),
         ("M", _i), ("K", _i), ("Ntok", _i), ("M0", _i), ("L", _i),
-        ("token_major", _i), ("out_dtype", _i), ("tile_n", _i),
+        ("token_major", _i), ("out_dtype", _i), ("tile_n", _i), ("schedule", _i),
     ]
 
 

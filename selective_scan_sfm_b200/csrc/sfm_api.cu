@@ -17,7 +17,7 @@ using namespace sfm;
 
 namespace {
 
-constexpr int kAbiVersion = 3;
+constexpr int kAbiVersion = 4;
 constexpr int kMaxDTile = 128;
 constexpr int kMaxChunk = 256;
 constexpr int kMaxB1 = 65535;  // grid.y
@@ -545,6 +545,7 @@ sfm_status sfm_proj_gemm(const sfm_proj_args* a, sfm_stream_t stream) {
   if (a->token_major ? (a->M0 != a->M || a->out1) : (a->M0 < 1 || a->M0 > a->M || ((a->M0 < a->M) != !!a->out1)))
     return SFM_ERR_INVALID_ARG;
   if (a->tile_n != 0 && a->tile_n != 128 && a->tile_n != 256) return SFM_ERR_UNSUPPORTED;
+  if (a->schedule < 0 || a->schedule > 2) return SFM_ERR_INVALID_ARG;
   if (a->K % 8 != 0) return SFM_ERR_UNSUPPORTED;  // TMA: the row pitch of W and X is a multiple of 16 bytes
   const void* ptrs[] = {a->W, a->X, a->out0, a->out1};
   for (const void* q : ptrs)
@@ -569,9 +570,13 @@ sfm_status sfm_proj_gemm(const sfm_proj_args* a, sfm_stream_t stream) {
   p.L = a->L;
   p.token_major = a->token_major;
   p.out_f32 = a->out_dtype == SFM_F32;
-  // 128 channels per tile for the short K of the projections (more, smaller CTAs: their
-  // epilogue stores overlap the others' loads), 256 when K is long and the MMAs dominate
-  p.bn = a->tile_n ? a->tile_n : (a->K > 640 ? 256 : 128);
+  // Short K (the projections): one CTA per tile of 128 channels, several CTAs per SM, so
+  // many warps store while others load -- the outputs' coalesced row stores bound these.
+  // Long K: the MMAs dominate; one persistent CTA per SM with tiles of 256 channels, its
+  // epilogue overlapping the next tile's loads and MMAs.
+  const bool long_k = a->K > 640;
+  p.bn = a->tile_n ? a->tile_n : (long_k ? 256 : 128);
+  p.persistent = a->schedule == 2 || (a->schedule == 0 && long_k);
   if (fault_injected()) return SFM_ERR_CUDA;
   return cuda_status(launch_proj(p, stream));
 }

@@ -66,6 +66,7 @@ struct ProjParams {
   int token_major;  // 1: out0 is [Ntok, M]
   int out_f32;      // 1: fp32 outputs, else bf16
   int bn;           // output channels per CTA tile: 128 or 256
+  int persistent;   // 1: one CTA per SM walks its tiles, epilogue overlapped with the next tile
 };
 
 struct BwdParams {

@@ -267,6 +267,214 @@ __global__ void __launch_bounds__(kThreads)
   }
 }
 
+// ------------------------------------------------------------------ persistent form
+//
+// One CTA per SM walks its tiles (tile t, t + gridDim.x, ...; the channel tile varies
+// fastest) with the work split by warp:
+//   warp 0  (one thread) TMA producer: keeps a ring of STAGES K-slices full across tiles;
+//   warp 1  (one thread) MMA issuer:   accumulates tile i in TMEM buffer i % 2;
+//   warps 2-9            epilogue:     drain buffer i % 2 into registers, hand it back to
+//                                      the MMA warp, then store while tile i + 1 accumulates.
+// Handshakes are mbarriers: full/empty per ring stage (TMA <-> MMA), acc_full/acc_empty per
+// accumulator (MMA <-> epilogue).  Every wait is bounded; a wait that gives up records
+// SFM_ERR_TIMEOUT, every role leaves its loop, the MMA warp drains its own MMAs and the
+// producer its own copies (both bounded), and the tensor memory is freed.
+constexpr int kPThreads = 320;
+
+template <int NT, int STAGES>
+struct PSmem {
+  static constexpr int kStageA = kBM * kBK * 2;
+  static constexpr int kStageB = NT * kBK * 2;
+  static constexpr int kRing = STAGES * (kStageA + kStageB);
+  static constexpr int kBars = (2 * STAGES + 5) * 8 + 16;
+  static constexpr int kBytes = 1024 + kRing + kBars;
+};
+
+template <int NT, int STAGES, typename TO>
+__global__ void __launch_bounds__(kPThreads, 1)
+    proj_gemm_persistent(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                         const ProjParams p) {
+  using SM = PSmem<NT, STAGES>;
+  extern __shared__ __align__(16) char smem_raw[];
+  char* ring = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(ring + SM::kRing);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;   // [2]
+  uint64_t* drain = acc_empty + 2;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(drain + 1) + 1;
+  auto stage_a = [&](int s) { return ring + s * SM::kStageA; };
+  auto stage_b = [&](int s) { return ring + STAGES * SM::kStageA + s * SM::kStageB; };
+  auto give_up = [&]() {
+    atomicExch(&g_proj_error, (unsigned)SFM_ERR_TIMEOUT);
+    *abort_flag = 1;
+  };
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_ct = (p.M + NT - 1) / NT, n_tt = (p.Ntok + kBM - 1) / kBM;
+  const int ntiles = n_ct * n_tt;
+  const int nk = (p.K + kBK - 1) / kBK;
+
+  if (tid == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], 8);  // one arrival per epilogue warp
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 0) {  // two accumulators of NT fp32 columns x 128 lanes
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                     smem_u32(const_cast<uint32_t*>(tmem_slot))),
+                 "r"((uint32_t)(2 * NT))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {  // ---- producer
+      long long g = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x) {
+        const int n0 = (tile / n_ct) * kBM, c0 = (tile % n_ct) * NT;
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          const long long u = g / STAGES;
+          if (u >= 1 && !mbar_wait_bounded(&empty[s], (unsigned)((u - 1) & 1))) {
+            give_up();
+            break;
+          }
+          if (*abort_flag) break;
+          mbar_expect_tx(&full[s], (unsigned)(SM::kStageA + SM::kStageB));
+          tma_load_2d(stage_a(s), &tmX, kb * kBK, n0, &full[s]);
+          tma_load_2d(stage_b(s), &tmW, kb * kBK, c0, &full[s]);
+        }
+      }
+      if (*abort_flag)  // let the copies still in flight land before the CTA leaves
+        for (long long q = g > STAGES ? g - STAGES : 0; q < g; ++q)
+          mbar_wait_bounded(&full[q % STAGES], (unsigned)((q / STAGES) & 1));
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {  // ---- MMA issuer
+      const uint32_t idesc =
+          (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(NT >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+      long long g = 0;
+      int li = 0;
+      for (int tile = blockIdx.x; tile < ntiles && !*abort_flag; tile += gridDim.x, ++li) {
+        const int a = li & 1, use = li >> 1;
+        if (use >= 1 && !mbar_wait_bounded(&acc_empty[a], (unsigned)((use - 1) & 1))) {
+          give_up();
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + (uint32_t)(a * NT);
+        bool ok = true;
+        for (int kb = 0; kb < nk; ++kb, ++g) {
+          const int s = (int)(g % STAGES);
+          if (!mbar_wait_bounded(&full[s], (unsigned)((g / STAGES) & 1))) {
+            give_up();
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t da = kmajor_sw128_desc(smem_u32(stage_a(s)));
+          const uint64_t db = kmajor_sw128_desc(smem_u32(stage_b(s)));
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk)
+            umma_f16(acc, da + 2 * kk, db + 2 * kk, idesc, (kb | kk) != 0);
+          umma_commit(&empty[s]);
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[a]);
+      }
+      umma_commit(drain);  // every MMA issued above has completed once this arrives
+      if (!mbar_wait_bounded(drain, 0)) give_up();
+    }
+  } else {  // ---- epilogue: warps 2-9; warp w reads TMEM lane quarter w % 4, column half (w - 2) / 4
+    const int q = warp & 3, half = (warp - 2) >> 2;
+    int li = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++li) {
+      const int a = li & 1, use = li >> 1;
+      if (!mbar_wait_bounded_sleepy(&acc_full[a], (unsigned)(use & 1))) {
+        if (lane == 0) give_up();
+        break;
+      }
+      if (*abort_flag) break;
+      tc_fence_after();
+      float v[NT / 2];
+#pragma unroll
+      for (int j = 0; j < NT / 2; j += 32) {
+        float w[32];
+        tmem_ld_32x32(tmem + (uint32_t)(a * NT) + ((uint32_t)(q * 32) << 16) + (uint32_t)(half * (NT / 2) + j), w);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[j + i] = w[i];
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[a]);  // the accumulator may be overwritten now
+
+      const int n0 = (tile / n_ct) * kBM, cbase = (tile % n_ct) * NT + half * (NT / 2);
+      const int n = n0 + q * 32 + lane;
+      if (n >= p.Ntok) continue;
+      const int b = n / p.L, t = n - b * p.L;
+      const long long base0 = (long long)b * p.M0 * p.L + t;
+      const long long base1 = (long long)b * (p.M - p.M0) * p.L + t;
+      TO* out0 = static_cast<TO*>(p.out0);
+      TO* out1 = static_cast<TO*>(p.out1);
+      if (p.token_major) {
+        TO* dst = out0 + (size_t)n * p.M + cbase;
+        if (cbase + NT / 2 <= p.M && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+          constexpr int E = 16 / (int)sizeof(TO);
+#pragma unroll
+          for (int j = 0; j < NT / 2; j += E) {
+            uint32_t w[4];
+            if constexpr (sizeof(TO) == 2) {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(v[j + 2 * k], v[j + 2 * k + 1]);
+                w[k] = *reinterpret_cast<const uint32_t*>(&h);
+              }
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) w[k] = __float_as_uint(v[j + k]);
+            }
+            *reinterpret_cast<uint4*>(dst + j) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < NT / 2; ++j)
+            if (cbase + j < p.M) dst[j] = from_f<TO>(v[j]);
+        }
+      } else {  // one coalesced warp store per channel: 32 consecutive tokens of its row
+#pragma unroll
+        for (int j = 0; j < NT / 2; ++j) {
+          const int m = cbase + j;
+          if (m < p.M0)
+            out0[base0 + (long long)m * p.L] = from_f<TO>(v[j]);
+          else if (m < p.M)
+            out1[base1 + (long long)(m - p.M0) * p.L] = from_f<TO>(v[j]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"((uint32_t)(2 * NT))
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------------ host side
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -314,12 +522,34 @@ cudaError_t launch_nt(const ProjParams& p, const CUtensorMap& mx, const CUtensor
   return cudaGetLastError();
 }
 
+template <int NT, int STAGES, typename TO>
+cudaError_t launch_persistent(const ProjParams& p, const CUtensorMap& mx, const CUtensorMap& mw, cudaStream_t s) {
+  constexpr int bytes = PSmem<NT, STAGES>::kBytes;
+  static bool set = false;
+  if (!set) {
+    cudaError_t e = cudaFuncSetAttribute(proj_gemm_persistent<NT, STAGES, TO>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    set = true;
+  }
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long tiles = (long long)((p.M + NT - 1) / NT) * ((p.Ntok + kBM - 1) / kBM);
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  proj_gemm_persistent<NT, STAGES, TO><<<grid, kPThreads, bytes, s>>>(mx, mw, p);
+  return cudaGetLastError();
+}
+
 template <typename TO>
 cudaError_t launch_to(const ProjParams& p, cudaStream_t s) {
   CUtensorMap mx, mw;
   const int nt = p.bn <= 128 ? 128 : 256;
   if (!make_kmajor_map(&mx, p.X, p.Ntok, p.K, kBM) || !make_kmajor_map(&mw, p.W, p.M, p.K, nt))
     return cudaErrorInvalidValue;
+  if (p.persistent) {
+    if (nt == 128) return launch_persistent<128, 6, TO>(p, mx, mw, s);
+    return launch_persistent<256, 4, TO>(p, mx, mw, s);
+  }
   // K of at most 10 stages: a 2-stage ring, so several CTAs share an SM and one's epilogue
   // overlaps the others' loads and MMAs; longer K: 4 stages
   const bool short_k = p.K <= 10 * kBK;

@@ -32,7 +32,7 @@ def test_exports_every_declared_symbol(L):
 
 
 def test_status_strings_and_version(L):
-    assert L.sfm_abi_version() == 3
+    assert L.sfm_abi_version() == 4
     for code in range(6):
         assert _abi.status_string(code).startswith("SFM_")
     assert _abi.status_string(99) == "SFM_ERR_UNKNOWN"
@@ -247,6 +247,7 @@ def proj_args(**kw):
     ("out1", None, _abi.SFM_ERR_INVALID_ARG),       # M0 < M needs the second output
     ("token_major", 1, _abi.SFM_ERR_INVALID_ARG),   # token-major writes one output of all M rows
     ("tile_n", 64, _abi.SFM_ERR_UNSUPPORTED),
+    ("schedule", 3, _abi.SFM_ERR_INVALID_ARG),
     ("out_dtype", 5, _abi.SFM_ERR_INVALID_ARG),
     ("X", FAKE + (1 << 24) + 8, _abi.SFM_ERR_MISALIGNED),
     ("out0", FAKE + (1 << 24), _abi.SFM_ERR_INVALID_ARG),  # output aliases X
@@ -260,6 +261,7 @@ def test_proj_valid_args_reach_the_launch_path(L, inject):
     assert L.sfm_proj_gemm(ctypes.byref(proj_args(token_major=1, M0=256, out1=None)), None) == _abi.SFM_ERR_CUDA
     assert L.sfm_proj_gemm(ctypes.byref(proj_args(M0=256, out1=None, tile_n=256, out_dtype=_abi.SFM_F32)),
                            None) == _abi.SFM_ERR_CUDA
+    assert L.sfm_proj_gemm(ctypes.byref(proj_args(schedule=2)), None) == _abi.SFM_ERR_CUDA
 
 
 def test_conv1d_tokens_validation(L, inject):

@@ -36,6 +36,10 @@ def check(got, ref, mag, dtype):
         assert err <= 1.0, err
 
 
+SCHEDULES = (1, 2)  # one CTA per tile; persistent
+
+
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("M,K,B,L,M0,tile_n,dt", [
     (128, 64, 2, 64, 128, 128, torch.float32),        # one CTA, one K step
     (256, 320, 4, 51, 128, 256, torch.bfloat16),      # in_proj shape: x and z split, ragged token tail
@@ -43,9 +47,9 @@ def check(got, ref, mag, dtype):
     (1280, 640, 8, 198, 640, 0, torch.bfloat16),      # stage-3 in_proj rows, automatic tile
     (64, 1280, 2, 51, 64, 256, torch.float32),        # long K (20 stages through a 4-stage ring)
 ])
-def test_channel_major(M, K, B, L, M0, tile_n, dt):
+def test_channel_major(M, K, B, L, M0, tile_n, dt, schedule):
     W, X = draw(M, K, B * L, seed=M + K + L)
-    o0, o1 = sfm_proj_gemm(W.cuda(), X.cuda(), L, M0=M0, out_dtype=dt, tile_n=tile_n)
+    o0, o1 = sfm_proj_gemm(W.cuda(), X.cuda(), L, M0=M0, out_dtype=dt, tile_n=tile_n, schedule=schedule)
     torch.cuda.synchronize()
     assert sfm_get_device_error(clear=True) == 0
     r0, r1 = oracle.proj(W.double().numpy(), X.double().numpy(), L, M0=M0)
@@ -57,10 +61,11 @@ def test_channel_major(M, K, B, L, M0, tile_n, dt):
         assert o1 is None
 
 
+@pytest.mark.parametrize("schedule", SCHEDULES)
 @pytest.mark.parametrize("M,K,Ntok,dt", [(40, 640, 198 * 3, torch.bfloat16), (72, 320, 300, torch.float32)])
-def test_token_major(M, K, Ntok, dt):
+def test_token_major(M, K, Ntok, dt, schedule):
     W, X = draw(M, K, Ntok, seed=M * 7 + K)
-    o, none = sfm_proj_gemm(W.cuda(), X.cuda(), 1, token_major=True, out_dtype=dt)
+    o, none = sfm_proj_gemm(W.cuda(), X.cuda(), 1, token_major=True, out_dtype=dt, schedule=schedule)
     assert none is None
     ref = oracle.proj(W.double().numpy(), X.double().numpy(), 1, token_major=True)
     check(o, ref, bound(W, X, 1, None, True), dt)
