@@ -147,6 +147,14 @@ def write_lut(results, path=LUT, gpu=None):
     open(path, "w").write("\n".join(lines) + "\n")
 
 
+def merge(base, newer):
+    """The rows of `base` with those of the same (T, B, D, N) replaced by `newer`'s, in base order."""
+    key = lambda r: (r["T"], r["B"], r["D"], r["N"])
+    fresh = {key(r): r for r in newer}
+    out = [fresh.pop(key(r), r) for r in base]
+    return out + list(fresh.values())
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--quick", action="store_true")
@@ -154,17 +162,26 @@ def main():
     ap.add_argument("--json", default=None)
     ap.add_argument("--reps", type=int, default=15)
     ap.add_argument("--from-json", default=None, help="rewrite the table from a saved sweep (no GPU needed)")
+    ap.add_argument("--T", type=int, default=None, help="sweep only the shapes of this patch-token count")
+    ap.add_argument("--merge", default=None,
+                    help="a saved full sweep whose rows for the swept shapes are replaced before writing")
     a = ap.parse_args()
     if a.from_json:
-        write_lut(json.load(open(a.from_json)))
+        rows = json.load(open(a.from_json))
+        if a.merge:
+            rows = merge(json.load(open(a.merge)), rows)
+        write_lut(rows)
         return
-    res = sweep(GRID_QUICK if a.quick else GRID_FULL, reps=a.reps)
+    grid = GRID_QUICK if a.quick else GRID_FULL
+    if a.T is not None:
+        grid = [g for g in grid if g[0] == a.T]
+    res = sweep(grid, reps=a.reps)
     for r in res:
         r["gpu"] = torch.cuda.get_device_name()
     if a.json:
         json.dump(res, open(a.json, "w"), indent=1)
     if a.write:
-        write_lut(res)
+        write_lut(merge(json.load(open(a.merge)), res) if a.merge else res)
 
 
 if __name__ == "__main__":
