@@ -485,6 +485,42 @@ def measure_proj(steps, warmup, world, device, workload="stage4_t49", seed=0):
     return out
 
 
+def measure_bwd(steps, warmup, world, device, workload="chain4_stage3", seed_base=0):
+    """The backward of the whole mixer layer (aux init, conv + SiLU, folded scan, gate,
+    swap) at a workload's layer shape, timed alone over rotating input sets."""
+    import torch
+    from selective_scan_sfm_b200 import _abi, _mixer_bwd_args, synth
+
+    w = synth.WORKLOADS[workload]
+    B, D, T, N, K = w["B"], w["D"], w["T"], w["N"], w["K"]
+    L = T + 2
+    esz = 2 if w["dtype"] == "bf16" else 4
+    # inputs read (x, dt, z, B, C, dout) and fp32 gradients written (dx, ddt, dz, dB, dC)
+    set_bytes = B * D * (T + 3 * L) * esz + 2 * B * N * L * esz + B * D * (T + 2 * L) * 4 + 2 * B * N * L * 4
+    nsets = max(2, math.ceil(2 * L2_BYTES / set_bytes) + 1)
+    stream = torch.cuda.current_stream(device)
+    sp = ctypes.c_void_p(stream.cuda_stream)
+    lib = _abi.lib()
+    keep, cargs = [], []
+    for i in range(nsets):
+        d = synth.make_inputs(**w, seed=seed_base + 13 * i)
+        dc = {k: (v.to(device) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+        dout = synth.make_dout(B, D, L, seed=seed_base + i).to(device)
+        a, g, grads, ws = _mixer_bwd_args(dc["x"], dc["dt"], dc["Bm"], dc["Cm"], dc["A"], dout, dc["z"], dc["Dskip"],
+                                          dc["dt_bias"], dc["conv_w"], dc["conv_b"], None, True, True, True, None)
+        keep.append((dc, dout, grads, ws))
+        cargs.append((a, g, ctypes.c_void_p(ws.data_ptr()), ws.numel()))
+
+    def launch(i):
+        a, g, wp, wn = cargs[i % nsets]
+        rc = lib.sfm_mixer_bwd(ctypes.byref(a), ctypes.byref(g), wp, wn, sp)
+        if rc != 0:
+            raise RuntimeError(_abi.status_string(rc))
+
+    total_ms, _ = _time_launches(launch, nsets, steps, warmup, world, device, stream)
+    return dict(ms=total_ms / steps, elements=B * D * L, bytes=set_bytes, workspace=cargs[0][3], w=w)
+
+
 def max_over_ranks(v, world, device):
     if world == 1:
         return v
@@ -570,6 +606,17 @@ def main(argv=None):
                                            "padded to the longest (%d of %d elements useful)"
                                            % (rr["elements"], rr["padded_elements"])}}
 
+    bwd = {}
+    if not args.no_extra:
+        rb = measure_bwd(args.steps, args.warmup, world, device, seed_base=1000 * rank)
+        bms = max_over_ranks(rb["ms"], world, device)
+        bwd = {"workload": "chain4_stage3 layer (B=64, D=640, T=196+2, N=16, bf16): sfm_mixer_bwd, all gradients",
+               "value": world * rb["elements"] / (bms * 1e-3), "unit": "elems/s", "ms_per_step": bms,
+               "hbm": {"achieved": rb["bytes"] / (bms * 1e-3) / 1e9, "unit": "GB/s",
+                       "note": "inputs read and fp32 gradients written once; the %.0f MB workspace "
+                               "(the forward states the reverse sweep reads back) not counted"
+                               % (rb["workspace"] / 1e6)}}
+
     proj = {}
     if not args.no_extra:
         pr = measure_proj(args.steps, args.warmup, world, device)
@@ -639,6 +686,9 @@ def main(argv=None):
         line["t196"] = extra
     if ragged:
         line["ragged"] = ragged
+    if bwd:
+        bwd["hbm"].update(peak=hbm_peak, frac=bwd["hbm"]["achieved"] / hbm_peak)
+        line["bwd"] = bwd
     if proj:
         bf_peak = float(peaks.get("bf16_tflops", 1590.0)) if peaks else 1590.0
         bf_sus = float(peaks.get("bf16_tflops_sustained", 1400.0)) if peaks else 1400.0

@@ -341,11 +341,8 @@ def sfm_selective_scan_fold_bwd_noalloc(u, dt, Bm, Cm, A, dout, grads, *, z=None
     return grads
 
 
-def sfm_mixer_bwd(x, dt, Bm, Cm, A, dout, *, z=None, Dskip=None, dt_bias=None, conv_w=None, conv_b=None,
-                  pad_left=None, dt_softplus=True, aux_init=False, swap_out=False, workspace=None, stream=None):
-    """Backward of the whole fused layer (same arguments as sfm_selective_scan_fold).
-    dout is the gradient of the stored output (after the swap).  Returns fp32 grads:
-    dx, dconv_w, dconv_b, ddt, dz, dA, dDskip, ddt_bias, dB, dC (those that apply)."""
+def _mixer_bwd_args(x, dt, Bm, Cm, A, dout, z, Dskip, dt_bias, conv_w, conv_b, pad_left, dt_softplus, aux_init,
+                    swap_out, workspace):
     a, _ = _scan_args(x, dt, Bm, Cm, A, z, Dskip, dt_bias, conv_w, conv_b, None, None, 0, pad_left, dt_softplus,
                       aux_init, swap_out, None, 0, 0, 0, need_y=False)
     B, D, L, N = a.B, a.D, a.L, a.N
@@ -375,6 +372,16 @@ def sfm_mixer_bwd(x, dt, Bm, Cm, A, dout, *, z=None, Dskip=None, dt_bias=None, c
     if workspace is None:
         workspace = torch.empty(max(int(need.value), 1), dtype=torch.uint8, device=dev)
     _dev(workspace, "workspace", torch.uint8)
+    return a, g, grads, workspace
+
+
+def sfm_mixer_bwd(x, dt, Bm, Cm, A, dout, *, z=None, Dskip=None, dt_bias=None, conv_w=None, conv_b=None,
+                  pad_left=None, dt_softplus=True, aux_init=False, swap_out=False, workspace=None, stream=None):
+    """Backward of the whole fused layer (same arguments as sfm_selective_scan_fold).
+    dout is the gradient of the stored output (after the swap).  Returns fp32 grads:
+    dx, dconv_w, dconv_b, ddt, dz, dA, dDskip, ddt_bias, dB, dC (those that apply)."""
+    a, g, grads, workspace = _mixer_bwd_args(x, dt, Bm, Cm, A, dout, z, Dskip, dt_bias, conv_w, conv_b, pad_left,
+                                             dt_softplus, aux_init, swap_out, workspace)
     _abi.check(_abi.lib().sfm_mixer_bwd(ctypes.byref(a), ctypes.byref(g), ctypes.c_void_p(workspace.data_ptr()),
                                         workspace.numel(), _stream(stream)), "sfm_mixer_bwd")
     return grads

@@ -9,11 +9,13 @@
 // previous state through that token.
 //
 // Schedule (built for exact, reproducible sums rather than speed):
-//   bwd_main_kernel: grid (channel tiles, B); one thread per channel loops over the N
-//     states.  Per state: a forward sweep stores h_t in the workspace, a reverse sweep
-//     accumulates du, dDelta and dA in the caller's fp32 outputs / registers and writes
-//     each channel's dB/dC contribution; the CTA then sums those over its channels in a
-//     fixed order into per-tile partials.
+//   bwd_main_kernel: grid (channel tiles, B); one thread per channel.  It first lays out
+//     u, Delta and the gated output gradient per token (once), then loops over the N
+//     states: a forward sweep stores h_t, a reverse sweep accumulates du, dDelta and dA
+//     and writes each channel's dB/dC contribution; the CTA then sums those over its
+//     channels in a fixed order into per-tile partials.  Every per-token array of the
+//     workspace is time-major [B, L, D], so the channels of a warp read and write one
+//     contiguous run per token; the caller's row-major outputs are written once at the end.
 //   bwd_reduce_bc_kernel: dB, dC = sum of the tile partials, in tile order.
 //   bwd_reduce_param_kernel: dA, dDskip, ddt_bias = sum over samples, in sample order.
 #include <mutex>
@@ -54,7 +56,6 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
   const size_t row = ((size_t)b * p.D + d) * L;
 
   const TI* u = MIXER ? nullptr : static_cast<const TI*>(p.u) + row;
-  const float* uw = MIXER ? p.u_ws + row : nullptr;
   const TI* dt = static_cast<const TI*>(p.dt) + row;
   const TI* z = gate ? static_cast<const TI*>(p.z) + row : nullptr;
   const TD* dout = static_cast<const TD*>(p.dout) + row;
@@ -63,11 +64,19 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
   const float dsk = p.Dskip ? p.Dskip[d] : 0.0f;
   const float dtb = p.dt_bias ? p.dt_bias[d] : 0.0f;
   float* du = p.du + row;
-  float* ddt = p.ddt + row;  // holds dLoss/dDelta until the final pass
-  float* dz = gate ? p.dz + row : nullptr;  // holds the pre-gate output y until the final pass
-  float* hb = p.hbuf + row;
-  float* cB = p.cB + row;
-  float* cC = p.cC + row;
+  float* ddt = p.ddt + row;
+  float* dz = gate ? p.dz + row : nullptr;
+  // time-major workspace: element (b, t, this channel)
+  const size_t tm0 = (size_t)b * L * p.D + d, tD = (size_t)p.D;
+  float* tu = p.tm_u + tm0;
+  float* tdl = p.tm_dl + tm0;   // Delta_t
+  float* tgy = p.tm_gy + tm0;   // dLoss/dy_t through the gate
+  float* tdu = p.tm_du + tm0;   // dLoss/du_t, accumulated over the states
+  float* tdd = p.tm_dd + tm0;   // dLoss/dDelta_t, accumulated over the states
+  float* ty = p.tm_y + tm0;     // the pre-gate output y_t (for dz)
+  float* hb = p.hbuf + tm0;
+  float* cB = p.cB + tm0;
+  float* cC = p.cC + tm0;
 
   auto delta_at = [&](int t) {
     const float v = to_f(dt[t]) + dtb;
@@ -78,27 +87,30 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
     const int i = (MIXER && p.swap_dout) ? (t == 0 ? L - 1 : (t == L - 1 ? 0 : t)) : t;
     return to_f(dout[i]);
   };
-  auto gy_at = [&](int t) { return gate ? dout_at(t) * silu(to_f(z[t])) : dout_at(t); };
-  auto u_at = [&](int t) { return MIXER ? uw[t] : to_f(u[t]); };
 
-  if (MIXER && active) {  // the scan input of the layer, once: u = SiLU(conv(xa)) (or xa without conv)
-    const TI* xr = static_cast<const TI*>(p.x) + ((size_t)b * p.D + d) * p.Tx;
+  // per token, once: u (the layer's scan input, u = SiLU(conv(xa)) in mixer mode), Delta
+  // and the output gradient through the gate, each laid out time-major
+  float sum_dsk = 0.0f;
+  if (active) {
+    const TI* xr = MIXER ? static_cast<const TI*>(p.x) + ((size_t)b * p.D + d) * p.Tx : nullptr;
     float mean = 0.0f;
-    if (p.aux) {
+    if (MIXER && p.aux) {
       for (int t = 0; t < p.Tx; ++t) mean += to_f(xr[t]);
       mean /= (float)p.Tx;
     }
-    float* uo = p.u_ws + row;
-    for (int t = 0; t < L; ++t) uo[t] = p.conv ? silu(conv_pre(p, xr, t, d, mean)) : xa_row(xr, t, L, p.aux, mean);
-  }
-
-  float sum_dsk = 0.0f;
-  if (active) {
     for (int t = 0; t < L; ++t) {
-      const float gy = gy_at(t), ut = u_at(t);
-      du[t] = gy * dsk;
-      ddt[t] = 0.0f;
-      if (gate) dz[t] = dsk * ut;
+      float ut;
+      if constexpr (MIXER)
+        ut = p.conv ? silu(conv_pre(p, xr, t, d, mean)) : xa_row(xr, t, L, p.aux, mean);
+      else
+        ut = to_f(u[t]);
+      const float gy = gate ? dout_at(t) * silu(to_f(z[t])) : dout_at(t);
+      tu[t * tD] = ut;
+      tdl[t * tD] = delta_at(t);
+      tgy[t * tD] = gy;
+      tdu[t * tD] = gy * dsk;
+      tdd[t * tD] = 0.0f;
+      if (gate) ty[t * tD] = dsk * ut;
       sum_dsk = fmaf(gy, ut, sum_dsk);
     }
   }
@@ -111,29 +123,29 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
       // forward sweep: h_t (the reset token starts from 0)
       float h = 0.0f;
       for (int t = 0; t < L; ++t) {
-        const float delta = delta_at(t);
-        const float bu = delta * to_f(Bn[t]) * u_at(t);
+        const float delta = tdl[t * tD];
+        const float bu = delta * to_f(Bn[t]) * tu[t * tD];
         h = t == 0 ? bu : fmaf(ex2(delta * an * kLog2e), h, bu);
-        hb[t] = h;
-        if (gate) dz[t] = fmaf(to_f(Cn[t]), h, dz[t]);
+        hb[t * tD] = h;
+        if (gate) ty[t * tD] = fmaf(to_f(Cn[t]), h, ty[t * tD]);
       }
       // reverse sweep
       float g = 0.0f, a_next = 0.0f, dA = 0.0f;
       for (int t = L - 1; t >= 0; --t) {
-        const float delta = delta_at(t), gy = gy_at(t), ut = u_at(t), Bv = to_f(Bn[t]);
+        const float delta = tdl[t * tD], gy = tgy[t * tD], ut = tu[t * tD], Bv = to_f(Bn[t]);
         g = fmaf(gy, to_f(Cn[t]), t + 1 < L ? a_next * g : 0.0f);
-        cC[t] = gy * hb[t];
-        cB[t] = g * delta * ut;
-        du[t] = fmaf(g * delta, Bv, du[t]);
+        cC[t * tD] = gy * hb[t * tD];
+        cB[t * tD] = g * delta * ut;
+        tdu[t * tD] = fmaf(g * delta, Bv, tdu[t * tD]);
         float dd = g * Bv * ut;
         float a_t = 0.0f;
         if (t > 0) {
           a_t = ex2(delta * an * kLog2e);
-          const float gha = g * hb[t - 1] * a_t;  // dLoss/dAbar_t * Abar_t
+          const float gha = g * hb[(t - 1) * tD] * a_t;  // dLoss/dAbar_t * Abar_t
           dd = fmaf(gha, an, dd);
           dA = fmaf(gha, delta, dA);
         }
-        ddt[t] += dd;
+        tdd[t * tD] += dd;
         a_next = a_t;
       }
       p.partA[((size_t)b * p.D + d) * N + n] = dA;
@@ -142,10 +154,10 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
     // this tile's share of dB[b,n,:] and dC[b,n,:], summed over its channels in order
     for (int t = tid; t < L; t += nthr) {
       float sb = 0.0f, sc = 0.0f;
-      const size_t base = ((size_t)b * p.D + d0) * L + t;
+      const size_t base = ((size_t)b * L + t) * p.D + d0;
       for (int c = 0; c < dcount; ++c) {
-        sb += p.cB[base + (size_t)c * L];
-        sc += p.cC[base + (size_t)c * L];
+        sb += p.cB[base + c];
+        sc += p.cC[base + c];
       }
       const size_t o = (((size_t)b * p.ntiles + tile) * 2) * N * L + (size_t)n * L + t;
       p.partBC[o] = sb;
@@ -154,16 +166,18 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
     __syncthreads();
   }
 
-  if (active) {
+  if (active) {  // the caller's row-major outputs, once
     float sum_bias = 0.0f;
     for (int t = 0; t < L; ++t) {
       const float v = to_f(dt[t]) + dtb;
-      const float ds = use_sp ? ddt[t] * (v > 20.0f ? 1.0f : sigmoid(v)) : ddt[t];
+      const float dd = tdd[t * tD];
+      const float ds = use_sp ? dd * (v > 20.0f ? 1.0f : sigmoid(v)) : dd;
       ddt[t] = ds;
+      du[t] = tdu[t * tD];
       sum_bias += ds;
       if (gate) {
         const float zt = to_f(z[t]), sg = sigmoid(zt);
-        dz[t] = dout_at(t) * dz[t] * (sg * (1.0f + zt * (1.0f - sg)));
+        dz[t] = dout_at(t) * ty[t * tD] * (sg * (1.0f + zt * (1.0f - sg)));
       }
     }
     p.partD[(size_t)b * p.D + d] = sum_dsk;
@@ -213,7 +227,7 @@ static size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
 size_t bwd_workspace_bytes(int B, int D, int L, int N, int d_tile) {
   const size_t bdl = (size_t)B * D * L, ntiles = (size_t)((D + d_tile - 1) / d_tile);
   size_t s = 0;
-  s += 3 * align256(bdl * 4);                           // hbuf, cB, cC
+  s += 9 * align256(bdl * 4);                           // hbuf, cB, cC, tm_u, tm_dl, tm_gy, tm_du, tm_dd, tm_y
   s += align256((size_t)B * ntiles * 2 * N * L * 4);    // partBC
   s += align256((size_t)B * D * N * 4);                 // partA
   s += 2 * align256((size_t)B * D * 4);                 // partD, partBias
@@ -231,6 +245,12 @@ void bwd_carve(BwdParams& p, char* ws) {
   p.hbuf = take(bdl * 4);
   p.cB = take(bdl * 4);
   p.cC = take(bdl * 4);
+  p.tm_u = take(bdl * 4);
+  p.tm_dl = take(bdl * 4);
+  p.tm_gy = take(bdl * 4);
+  p.tm_du = take(bdl * 4);
+  p.tm_dd = take(bdl * 4);
+  p.tm_y = take(bdl * 4);
   p.partBC = take((size_t)p.B * p.ntiles * 2 * p.N * p.L * 4);
   p.partA = take((size_t)p.B * p.D * p.N * 4);
   p.partD = take((size_t)p.B * p.D * 4);

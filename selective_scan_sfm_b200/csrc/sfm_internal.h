@@ -80,8 +80,10 @@ struct BwdParams {
   const float* Dskip;
   const float* dt_bias;
   float *du, *ddt, *dz, *dA, *dDskip, *ddt_bias, *dB, *dC;
-  // workspace regions (carved by bwd_carve)
+  // workspace regions (carved by bwd_carve); hbuf, cB, cC and the tm_* arrays are
+  // time-major [B, L, D], so the channels of a warp touch one contiguous run per token
   float *hbuf, *cB, *cC, *partBC, *partA, *partD, *partBias;
+  float *tm_u, *tm_dl, *tm_gy, *tm_du, *tm_dd, *tm_y;
   int B, D, L, N, d_tile, ntiles;
   int softplus;
   // mixer mode (the whole layer): the scan input u = SiLU(conv(xa)) is built from x into
