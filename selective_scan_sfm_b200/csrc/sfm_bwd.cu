@@ -43,6 +43,11 @@ __device__ __forceinline__ float conv_pre(const BwdParams& p, const TI* xr, int 
   return acc;
 }
 
+static int bwd_fast_smem(int N, int L, int d_tile) {
+  // bc [L][2N] + red: 2 tokens x 2N rows of d_tile + 1 (the pad keeps the row sums off one bank)
+  return (int)(((size_t)L * 2 * N + (size_t)2 * 2 * N * (d_tile + 1)) * sizeof(float));
+}
+
 template <typename TI, typename TD, bool MIXER>
 __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
   const int tid = threadIdx.x, nthr = blockDim.x;
@@ -185,6 +190,200 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
   }
 }
 
+// The same backward with all N (<= 16) states in registers: after the per-token prologue,
+// ONE forward sweep over the tokens computes every state's h_t (stored [B, L, N, D], so a
+// warp's channels store one contiguous run per (token, state)) and the pre-gate output,
+// and ONE reverse sweep carries every state's adjoint.  B and C of the sample are staged
+// in shared memory as fp32 [t][2N].  Each token's dB/dC contributions go to a shared
+// buffer of kRedT tokens, summed over the tile's channels in channel order when it fills.
+// Every sum runs in the order of bwd_main_kernel, so both give the same bits.
+constexpr int kFastN = 16, kRedT = 2;
+
+template <typename TI, typename TD, bool MIXER>
+__global__ void __launch_bounds__(64) bwd_fast_kernel(const BwdParams p) {
+  extern __shared__ float bsm[];
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int tile = blockIdx.x, b = blockIdx.y;
+  const int d0 = tile * p.d_tile;
+  const int dcount = min(p.d_tile, p.D - d0);
+  const bool active = tid < dcount;
+  const int d = d0 + (active ? tid : 0);
+  const int L = p.L, N = p.N, N2 = 2 * p.N;
+  const bool gate = p.z != nullptr, use_sp = p.softplus;
+  const size_t row = ((size_t)b * p.D + d) * L;
+  float* bc = bsm;                         // [L][2N]: B then C of token t
+  float* red = bsm + (size_t)L * N2;       // [kRedT][2N][d_tile + 1]
+  const int rstride = p.d_tile + 1;
+
+  const TI* u = MIXER ? nullptr : static_cast<const TI*>(p.u) + row;
+  const TI* dt = static_cast<const TI*>(p.dt) + row;
+  const TI* z = gate ? static_cast<const TI*>(p.z) + row : nullptr;
+  const TD* dout = static_cast<const TD*>(p.dout) + row;
+  const TI* Bm = static_cast<const TI*>(p.Bm) + (size_t)b * N * L;
+  const TI* Cm = static_cast<const TI*>(p.Cm) + (size_t)b * N * L;
+  const float dsk = p.Dskip ? p.Dskip[d] : 0.0f;
+  const float dtb = p.dt_bias ? p.dt_bias[d] : 0.0f;
+  float* du = p.du + row;
+  float* ddt = p.ddt + row;
+  float* dz = gate ? p.dz + row : nullptr;
+  const size_t tm0 = (size_t)b * L * p.D + d, tD = (size_t)p.D;
+  float* tu = p.tm_u + tm0;
+  float* tdl = p.tm_dl + tm0;
+  float* tgy = p.tm_gy + tm0;
+  float* tdu = p.tm_du + tm0;
+  float* tdd = p.tm_dd + tm0;
+  float* ty = p.tm_y + tm0;
+  float* hs = p.hstore + (size_t)b * L * N * p.D + d;  // h of (t, n) at hs[(t * N + n) * D]
+
+  for (int e = tid; e < L * N2; e += nthr) {
+    const int t = e / N2, j = e - t * N2;
+    bc[e] = j < N ? to_f(Bm[(size_t)j * L + t]) : to_f(Cm[(size_t)(j - N) * L + t]);
+  }
+  auto delta_at = [&](int t) {
+    const float v = to_f(dt[t]) + dtb;
+    return use_sp ? softplus(v) : v;
+  };
+  auto dout_at = [&](int t) {
+    const int i = (MIXER && p.swap_dout) ? (t == 0 ? L - 1 : (t == L - 1 ? 0 : t)) : t;
+    return to_f(dout[i]);
+  };
+  float sum_dsk = 0.0f;
+  if (active) {
+    const TI* xr = MIXER ? static_cast<const TI*>(p.x) + ((size_t)b * p.D + d) * p.Tx : nullptr;
+    float mean = 0.0f;
+    if (MIXER && p.aux) {
+      for (int t = 0; t < p.Tx; ++t) mean += to_f(xr[t]);
+      mean /= (float)p.Tx;
+    }
+#pragma unroll 2
+    for (int t = 0; t < L; ++t) {
+      float ut;
+      if constexpr (MIXER)
+        ut = p.conv ? silu(conv_pre(p, xr, t, d, mean)) : xa_row(xr, t, L, p.aux, mean);
+      else
+        ut = to_f(u[t]);
+      const float gy = gate ? dout_at(t) * silu(to_f(z[t])) : dout_at(t);
+      tu[t * tD] = ut;
+      tdl[t * tD] = delta_at(t);
+      tgy[t * tD] = gy;
+      tdu[t * tD] = gy * dsk;
+      tdd[t * tD] = 0.0f;
+      if (gate) ty[t * tD] = dsk * ut;
+      sum_dsk = fmaf(gy, ut, sum_dsk);
+    }
+  }
+  __syncthreads();
+
+  float An[kFastN];
+#pragma unroll
+  for (int n = 0; n < kFastN; ++n) An[n] = n < N ? p.A[(size_t)d * N + n] : 0.0f;
+
+  // forward sweep: every state's h_t, and the pre-gate output for dz
+  if (active) {
+    float h[kFastN];
+    const size_t hstep = (size_t)N * tD;  // h of the next token
+    float* hp = hs;
+    const float *pdl = tdl, *pu = tu;
+    float* py = ty;
+    const float* bt = bc;
+    for (int t = 0; t < L; ++t, hp += hstep, pdl += tD, pu += tD, py += tD, bt += N2) {
+      const float delta = *pdl, ut = *pu;
+      float yv = gate ? *py : 0.0f;
+#pragma unroll
+      for (int n = 0; n < kFastN; ++n) {
+        if (n < N) {
+          const float bu = delta * bt[n] * ut;
+          h[n] = t == 0 ? bu : fmaf(ex2(delta * An[n] * kLog2e), h[n], bu);
+          hp[n * tD] = h[n];
+          if (gate) yv = fmaf(bt[N + n], h[n], yv);
+        }
+      }
+      if (gate) *py = yv;
+    }
+  }
+
+  // reverse sweep: every state's adjoint; the dB/dC contributions through the buffer
+  float g[kFastN], a_next[kFastN], dA[kFastN];
+#pragma unroll
+  for (int n = 0; n < kFastN; ++n) g[n] = a_next[n] = dA[n] = 0.0f;
+  const size_t pbc = (((size_t)b * p.ntiles + tile) * 2) * N * L;
+  const size_t hstep = (size_t)N * tD;
+  for (int t = L - 1; t >= 0; --t) {
+    const int slot = (L - 1 - t) % kRedT;
+    if (active) {
+      const size_t o = (size_t)t * tD;
+      const float delta = tdl[o], gy = tgy[o], ut = tu[o];
+      const float* bt = bc + (size_t)t * N2;
+      const float* hp = hs + (size_t)t * hstep;          // h_t
+      const float* hq = t > 0 ? hp - hstep : hp;         // h_(t-1) (read only when t > 0)
+      float duv = tdu[o], ddv = tdd[o];
+      float* rs = red + (size_t)slot * N2 * rstride + tid;
+#pragma unroll
+      for (int n = 0; n < kFastN; ++n) {
+        if (n < N) {
+          const float Bv = bt[n], Cv = bt[N + n];
+          g[n] = fmaf(gy, Cv, t + 1 < L ? a_next[n] * g[n] : 0.0f);
+          rs[(N + n) * rstride] = gy * hp[n * tD];
+          rs[n * rstride] = g[n] * delta * ut;
+          duv = fmaf(g[n] * delta, Bv, duv);
+          float dd = g[n] * Bv * ut;
+          float a_t = 0.0f;
+          if (t > 0) {
+            a_t = ex2(delta * An[n] * kLog2e);
+            const float gha = g[n] * hq[n * tD] * a_t;
+            dd = fmaf(gha, An[n], dd);
+            dA[n] = fmaf(gha, delta, dA[n]);
+          }
+          ddv += dd;
+          a_next[n] = a_t;
+        }
+      }
+      tdu[o] = duv;
+      tdd[o] = ddv;
+    }
+    if (slot == kRedT - 1 || t == 0) {  // the buffered tokens t .. t + slot: sum over channels in order
+      __syncthreads();
+      for (int e = tid; e < (slot + 1) * N2; e += nthr) {
+        const int k = e / N2, j = e - k * N2;  // buffer slot k holds token t + slot - k
+        const float* r = red + ((size_t)k * N2 + j) * rstride;
+        float sum = 0.0f;
+        for (int c = 0; c < dcount; ++c) sum += r[c];
+        const int tt = t + slot - k;
+        p.partBC[pbc + (j < N ? (size_t)j * L : (size_t)N * L + (size_t)(j - N) * L) + tt] = sum;
+      }
+      __syncthreads();
+    }
+  }
+
+  if (active) {
+#pragma unroll
+    for (int n = 0; n < kFastN; ++n)
+      if (n < N) p.partA[((size_t)b * p.D + d) * N + n] = dA[n];
+    float sum_bias = 0.0f;
+#pragma unroll 4
+    for (int t = 0; t < L; ++t) {
+      const float v = to_f(dt[t]) + dtb;
+      const float dd = tdd[t * tD];
+      const float ds = use_sp ? dd * (v > 20.0f ? 1.0f : sigmoid(v)) : dd;
+      ddt[t] = ds;
+      du[t] = tdu[t * tD];
+      sum_bias += ds;
+      if (gate) {
+        const float zt = to_f(z[t]), sg = sigmoid(zt);
+        dz[t] = dout_at(t) * ty[t * tD] * (sg * (1.0f + zt * (1.0f - sg)));
+      }
+    }
+    p.partD[(size_t)b * p.D + d] = sum_dsk;
+    p.partBias[(size_t)b * p.D + d] = sum_bias;
+  }
+}
+
+// The register-resident kernel covers N <= 16 with B and C of a sample in 64 KB of
+// shared memory; other shapes take bwd_main_kernel.
+static bool bwd_fast_ok(int N, int L, int d_tile) {
+  return N <= kFastN && d_tile <= 64 && bwd_fast_smem(N, L, d_tile) <= 64 * 1024;
+}
+
 // dB[b,n,t] / dC[b,n,t]: sum over channel tiles in tile order.
 __global__ void bwd_reduce_bc_kernel(const BwdParams p) {
   const size_t NL = (size_t)p.N * p.L;
@@ -228,6 +427,7 @@ size_t bwd_workspace_bytes(int B, int D, int L, int N, int d_tile) {
   const size_t bdl = (size_t)B * D * L, ntiles = (size_t)((D + d_tile - 1) / d_tile);
   size_t s = 0;
   s += 9 * align256(bdl * 4);                           // hbuf, cB, cC, tm_u, tm_dl, tm_gy, tm_du, tm_dd, tm_y
+  if (bwd_fast_ok(N, L, d_tile)) s += align256(bdl * N * 4);  // hstore
   s += align256((size_t)B * ntiles * 2 * N * L * 4);    // partBC
   s += align256((size_t)B * D * N * 4);                 // partA
   s += 2 * align256((size_t)B * D * 4);                 // partD, partBias
@@ -251,6 +451,7 @@ void bwd_carve(BwdParams& p, char* ws) {
   p.tm_du = take(bdl * 4);
   p.tm_dd = take(bdl * 4);
   p.tm_y = take(bdl * 4);
+  p.hstore = bwd_fast_ok(p.N, p.L, p.d_tile) ? take(bdl * p.N * 4) : nullptr;
   p.partBC = take((size_t)p.B * p.ntiles * 2 * p.N * p.L * 4);
   p.partA = take((size_t)p.B * p.D * p.N * 4);
   p.partD = take((size_t)p.B * p.D * 4);
@@ -282,11 +483,28 @@ cudaError_t noalloc_scratch(void** out) {
   return cudaSuccess;
 }
 
+template <typename TI, typename TD, bool MIXER>
+static cudaError_t launch_main(const BwdParams& p, cudaStream_t s) {
+  const int threads = (p.d_tile + 31) & ~31;
+  if (p.hstore) {
+    const int bytes = bwd_fast_smem(p.N, p.L, p.d_tile);
+    static int have = 48 * 1024;
+    if (bytes > have) {
+      cudaError_t e = cudaFuncSetAttribute(bwd_fast_kernel<TI, TD, MIXER>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
+      if (e != cudaSuccess) return e;
+      have = 64 * 1024;
+    }
+    bwd_fast_kernel<TI, TD, MIXER><<<dim3(p.ntiles, p.B), threads, bytes, s>>>(p);
+  } else {
+    bwd_main_kernel<TI, TD, MIXER><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
 template <typename TI, typename TD>
 static cudaError_t launch_bwd_t(const BwdParams& p, cudaStream_t s) {
-  const int threads = (p.d_tile + 31) & ~31;
-  bwd_main_kernel<TI, TD, false><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_main<TI, TD, false>(p, s);
   if (e != cudaSuccess) return e;
   const size_t nbc = (size_t)p.B * p.N * p.L;
   bwd_reduce_bc_kernel<<<(unsigned)((nbc + 255) / 256), 256, 0, s>>>(p);
@@ -399,9 +617,7 @@ void mixer_bwd_carve(BwdParams& p, char* ws) {
 
 template <typename TI, typename TD>
 static cudaError_t launch_mixer_bwd_t(const BwdParams& p, cudaStream_t s) {
-  const int threads = (p.d_tile + 31) & ~31;
-  bwd_main_kernel<TI, TD, true><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_main<TI, TD, true>(p, s);
   if (e != cudaSuccess) return e;
   const size_t nbc = (size_t)p.B * p.N * p.L;
   bwd_reduce_bc_kernel<<<(unsigned)((nbc + 255) / 256), 256, 0, s>>>(p);

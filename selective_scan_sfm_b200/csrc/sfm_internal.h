@@ -84,6 +84,7 @@ struct BwdParams {
   // time-major [B, L, D], so the channels of a warp touch one contiguous run per token
   float *hbuf, *cB, *cC, *partBC, *partA, *partD, *partBias;
   float *tm_u, *tm_dl, *tm_gy, *tm_du, *tm_dd, *tm_y;
+  float* hstore;    // [B, L, N, D]: the forward states, for the register-resident kernel
   int B, D, L, N, d_tile, ntiles;
   int softplus;
   // mixer mode (the whole layer): the scan input u = SiLU(conv(xa)) is built from x into
