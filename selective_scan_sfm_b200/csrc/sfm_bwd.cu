@@ -283,12 +283,18 @@ __global__ void __launch_bounds__(64) bwd_fast_kernel(const BwdParams p) {
     float h[kFastN];
     const size_t hstep = (size_t)N * tD;  // h of the next token
     float* hp = hs;
-    const float *pdl = tdl, *pu = tu;
-    float* py = ty;
     const float* bt = bc;
-    for (int t = 0; t < L; ++t, hp += hstep, pdl += tD, pu += tD, py += tD, bt += N2) {
-      const float delta = *pdl, ut = *pu;
-      float yv = gate ? *py : 0.0f;
+    // the next token's inputs are loaded one step ahead
+    float nd = tdl[0], nu = tu[0], ny = gate ? ty[0] : 0.0f;
+    for (int t = 0; t < L; ++t, hp += hstep, bt += N2) {
+      const float delta = nd, ut = nu;
+      float yv = ny;
+      if (t + 1 < L) {
+        const size_t o = (size_t)(t + 1) * tD;
+        nd = tdl[o];
+        nu = tu[o];
+        if (gate) ny = ty[o];
+      }
 #pragma unroll
       for (int n = 0; n < kFastN; ++n) {
         if (n < N) {
@@ -298,7 +304,7 @@ __global__ void __launch_bounds__(64) bwd_fast_kernel(const BwdParams p) {
           if (gate) yv = fmaf(bt[N + n], h[n], yv);
         }
       }
-      if (gate) *py = yv;
+      if (gate) ty[(size_t)t * tD] = yv;
     }
   }
 
@@ -308,29 +314,54 @@ __global__ void __launch_bounds__(64) bwd_fast_kernel(const BwdParams p) {
   for (int n = 0; n < kFastN; ++n) g[n] = a_next[n] = dA[n] = 0.0f;
   const size_t pbc = (((size_t)b * p.ntiles + tile) * 2) * N * L;
   const size_t hstep = (size_t)N * tD;
+  // h_t and h_(t-1) are in registers; h_(t-2) and the next token's inputs load one step ahead
+  float hc[kFastN], hq[kFastN];
+  float nd = 0.0f, ngy = 0.0f, nu = 0.0f, ndu = 0.0f, ndd = 0.0f;
+  if (active) {
+    const size_t o = (size_t)(L - 1) * tD;
+    nd = tdl[o];
+    ngy = tgy[o];
+    nu = tu[o];
+    ndu = tdu[o];
+    ndd = tdd[o];
+#pragma unroll
+    for (int n = 0; n < kFastN; ++n) {
+      hc[n] = n < N ? hs[(size_t)(L - 1) * hstep + n * tD] : 0.0f;
+      hq[n] = (n < N && L > 1) ? hs[(size_t)(L - 2) * hstep + n * tD] : 0.0f;
+    }
+  }
   for (int t = L - 1; t >= 0; --t) {
     const int slot = (L - 1 - t) % kRedT;
     if (active) {
       const size_t o = (size_t)t * tD;
-      const float delta = tdl[o], gy = tgy[o], ut = tu[o];
+      const float delta = nd, gy = ngy, ut = nu;
+      float duv = ndu, ddv = ndd;
+      float hn[kFastN];  // h_(t-2), for the next step
+      if (t >= 1) {
+        const size_t o1 = (size_t)(t - 1) * tD;
+        nd = tdl[o1];
+        ngy = tgy[o1];
+        nu = tu[o1];
+        ndu = tdu[o1];
+        ndd = tdd[o1];
+      }
+#pragma unroll
+      for (int n = 0; n < kFastN; ++n) hn[n] = (n < N && t >= 2) ? hs[(size_t)(t - 2) * hstep + n * tD] : 0.0f;
       const float* bt = bc + (size_t)t * N2;
-      const float* hp = hs + (size_t)t * hstep;          // h_t
-      const float* hq = t > 0 ? hp - hstep : hp;         // h_(t-1) (read only when t > 0)
-      float duv = tdu[o], ddv = tdd[o];
       float* rs = red + (size_t)slot * N2 * rstride + tid;
 #pragma unroll
       for (int n = 0; n < kFastN; ++n) {
         if (n < N) {
           const float Bv = bt[n], Cv = bt[N + n];
           g[n] = fmaf(gy, Cv, t + 1 < L ? a_next[n] * g[n] : 0.0f);
-          rs[(N + n) * rstride] = gy * hp[n * tD];
+          rs[(N + n) * rstride] = gy * hc[n];
           rs[n * rstride] = g[n] * delta * ut;
           duv = fmaf(g[n] * delta, Bv, duv);
           float dd = g[n] * Bv * ut;
           float a_t = 0.0f;
           if (t > 0) {
             a_t = ex2(delta * An[n] * kLog2e);
-            const float gha = g[n] * hq[n * tD] * a_t;
+            const float gha = g[n] * hq[n] * a_t;
             dd = fmaf(gha, An[n], dd);
             dA[n] = fmaf(gha, delta, dA[n]);
           }
@@ -340,6 +371,11 @@ __global__ void __launch_bounds__(64) bwd_fast_kernel(const BwdParams p) {
       }
       tdu[o] = duv;
       tdd[o] = ddv;
+#pragma unroll
+      for (int n = 0; n < kFastN; ++n) {
+        hc[n] = hq[n];
+        hq[n] = hn[n];
+      }
     }
     if (slot == kRedT - 1 || t == 0) {  // the buffered tokens t .. t + slot: sum over channels in order
       __syncthreads();
