@@ -524,13 +524,9 @@ static cudaError_t launch_main(const BwdParams& p, cudaStream_t s) {
   const int threads = (p.d_tile + 31) & ~31;
   if (p.hstore) {
     const int bytes = bwd_fast_smem(p.N, p.L, p.d_tile);
-    static int have = 48 * 1024;
-    if (bytes > have) {
-      cudaError_t e = cudaFuncSetAttribute(bwd_fast_kernel<TI, TD, MIXER>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-      if (e != cudaSuccess) return e;
-      have = 64 * 1024;
-    }
+    static SmemLimit lim;
+    cudaError_t e = raise_smem_limit(bwd_fast_kernel<TI, TD, MIXER>, bytes, lim);
+    if (e != cudaSuccess) return e;
     bwd_fast_kernel<TI, TD, MIXER><<<dim3(p.ntiles, p.B), threads, bytes, s>>>(p);
   } else {
     bwd_main_kernel<TI, TD, MIXER><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);

@@ -1132,20 +1132,10 @@ int fwd_x_row(int chunk, int K, int esize) { return stage_row_bytes(chunk + K - 
 int fwd_io_row(int chunk, int esize) { return stage_row_bytes(chunk, esize); }
 int fwd_y_row(int chunk, int esize) { return out_row_bytes(chunk, esize); }
 
-// Raises the kernel's dynamic shared-memory limit to `bytes` when it is not yet that high.
-// `have` caches the limit already set (a race only repeats the same call).
-template <typename Kern>
-static cudaError_t set_smem(Kern k, int bytes, int& have) {
-  if (bytes <= have) return cudaSuccess;
-  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess) have = bytes;
-  return e;
-}
-
 template <typename TI, typename TO>
 static cudaError_t launch_lanes(const FwdParams& p, cudaStream_t s) {
-  static int have = 48 * 1024;
-  cudaError_t e = set_smem(fwd_lanes_kernel<TI, TO>, p.smem_bytes, have);
+  static SmemLimit lim;
+  cudaError_t e = raise_smem_limit(fwd_lanes_kernel<TI, TO>, p.smem_bytes, lim);
   if (e != cudaSuccess) return e;
   dim3 grid((p.D + p.d_tile - 1) / p.d_tile, p.B / p.B2);
   fwd_lanes_kernel<TI, TO><<<grid, p.d_tile * p.lanes, p.smem_bytes, s>>>(p);
@@ -1154,15 +1144,17 @@ static cudaError_t launch_lanes(const FwdParams& p, cudaStream_t s) {
 
 template <typename TI, typename TO, int NH, bool STD, int PE, int CPT>
 static cudaError_t launch_cpt(const FwdParams& p, cudaStream_t s) {
-  static int whole_set = 48 * 1024, chunk_set = 48 * 1024;
+  static SmemLimit whole_lim, chunk_lim;
   const int threads = ((p.d_tile + CPT - 1) / CPT + 31) & ~31;
   dim3 grid((p.D + p.d_tile - 1) / p.d_tile, p.B / p.B2);
   cudaError_t e;
   if (p.mode == kModeWhole) {
-    if ((e = set_smem(fwd_whole_kernel<TI, TO, NH, STD, PE, CPT>, p.smem_bytes, whole_set)) != cudaSuccess) return e;
+    if ((e = raise_smem_limit(fwd_whole_kernel<TI, TO, NH, STD, PE, CPT>, p.smem_bytes, whole_lim)) != cudaSuccess)
+      return e;
     fwd_whole_kernel<TI, TO, NH, STD, PE, CPT><<<grid, threads, p.smem_bytes, s>>>(p);
   } else {
-    if ((e = set_smem(fwd_chunk_kernel<TI, TO, NH, STD, PE, CPT>, p.smem_bytes, chunk_set)) != cudaSuccess) return e;
+    if ((e = raise_smem_limit(fwd_chunk_kernel<TI, TO, NH, STD, PE, CPT>, p.smem_bytes, chunk_lim)) != cudaSuccess)
+      return e;
     fwd_chunk_kernel<TI, TO, NH, STD, PE, CPT><<<grid, threads, p.smem_bytes, s>>>(p);
   }
   return cudaGetLastError();

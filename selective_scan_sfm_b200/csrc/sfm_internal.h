@@ -95,6 +95,25 @@ struct BwdParams {
   float *u_ws, *dx, *dconv_w, *dconv_b, *dw_part, *db_part;
 };
 
+// The dynamic shared-memory limit a kernel has been raised to, per device (the attribute
+// belongs to the function on each device).  raise_smem_limit calls cudaFuncSetAttribute
+// only when `bytes` exceeds what is recorded for the current device; on a device past the
+// table it always calls it.  A race between host threads only repeats the same call.
+struct SmemLimit {
+  int have[64] = {};  // 0: the default 48 KB
+};
+template <typename Kern>
+inline cudaError_t raise_smem_limit(Kern k, int bytes, SmemLimit& lim) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const bool cached = dev >= 0 && dev < 64;
+  if (cached && bytes <= (lim.have[dev] ? lim.have[dev] : 48 * 1024)) return cudaSuccess;
+  e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && cached) lim.have[dev] = bytes;
+  return e;
+}
+
 // Launchers (defined in the .cu files).  They only enqueue work; they return the
 // cudaError_t of the launch.
 cudaError_t launch_fwd(const FwdParams& p, sfm_dtype in_dtype, sfm_dtype out_dtype, int NP, cudaStream_t s);

@@ -510,13 +510,9 @@ bool make_kmajor_map(CUtensorMap* map, const void* base, long long rows, int K, 
 template <int NT, int STAGES, typename TO>
 cudaError_t launch_nt(const ProjParams& p, const CUtensorMap& mx, const CUtensorMap& mw, cudaStream_t s) {
   constexpr int bytes = ProjSmem<NT, STAGES>::kBytes;
-  static bool set = false;
-  if (!set) {
-    cudaError_t e = cudaFuncSetAttribute(proj_gemm_kernel<NT, STAGES, TO>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    set = true;
-  }
+  static SmemLimit lim;
+  cudaError_t e = raise_smem_limit(proj_gemm_kernel<NT, STAGES, TO>, bytes, lim);
+  if (e != cudaSuccess) return e;
   dim3 grid((p.Ntok + kBM - 1) / kBM, (p.M + NT - 1) / NT);
   proj_gemm_kernel<NT, STAGES, TO><<<grid, kThreads, bytes, s>>>(mx, mw, p);
   return cudaGetLastError();
@@ -525,13 +521,9 @@ cudaError_t launch_nt(const ProjParams& p, const CUtensorMap& mx, const CUtensor
 template <int NT, int STAGES, typename TO>
 cudaError_t launch_persistent(const ProjParams& p, const CUtensorMap& mx, const CUtensorMap& mw, cudaStream_t s) {
   constexpr int bytes = PSmem<NT, STAGES>::kBytes;
-  static bool set = false;
-  if (!set) {
-    cudaError_t e = cudaFuncSetAttribute(proj_gemm_persistent<NT, STAGES, TO>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    set = true;
-  }
+  static SmemLimit lim;
+  cudaError_t e = raise_smem_limit(proj_gemm_persistent<NT, STAGES, TO>, bytes, lim);
+  if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long tiles = (long long)((p.M + NT - 1) / NT) * ((p.Ntok + kBM - 1) / kBM);
