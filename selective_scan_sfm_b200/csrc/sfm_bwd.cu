@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
 constexpr int kFastN = 16, kRedT = 2;
 
 template <typename TI, typename TD, bool MIXER>
-__global__ void __launch_bounds__(64) bwd_fast_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(64, 5) bwd_fast_kernel(const BwdParams p) {
   extern __shared__ float bsm[];
   const int tid = threadIdx.x, nthr = blockDim.x;
   const int tile = blockIdx.x, b = blockIdx.y;
