@@ -8,8 +8,10 @@
 // section 3.3), so no gradient crosses samples and none flows into A, Delta or the
 // previous state through that token.
 //
-// Schedule (built for exact, reproducible sums rather than speed):
-//   bwd_main_kernel: grid (channel tiles, B); one thread per channel.  It first lays out
+// Schedule (every sum in a fixed order, so results are reproducible bit for bit):
+//   bwd_pair_kernel (N <= 16, B and C of a sample within 64 KB of shared memory): all
+//     states in registers, two threads per channel, one forward and one reverse sweep.
+//   bwd_main_kernel (other shapes): grid (channel tiles, B); one thread per channel.  It first lays out
 //     u, Delta and the gated output gradient per token (once), then loops over the N
 //     states: a forward sweep stores h_t, a reverse sweep accumulates du, dDelta and dA
 //     and writes each channel's dB/dC contribution; the CTA then sums those over its
@@ -190,29 +192,42 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
   }
 }
 
-// The same backward with all N (<= 16) states in registers: after the per-token prologue,
-// ONE forward sweep over the tokens computes every state's h_t (stored [B, L, N, D], so a
-// warp's channels store one contiguous run per (token, state)) and the pre-gate output,
-// and ONE reverse sweep carries every state's adjoint.  B and C of the sample are staged
-// in shared memory as fp32 [t][2N].  Each token's dB/dC contributions go to a shared
-// buffer of kRedT tokens, summed over the tile's channels in channel order when it fills.
-// Every sum runs in the order of bwd_main_kernel, so both give the same bits.
-constexpr int kFastN = 16, kRedT = 2;
+// The backward with all N (<= 16) states in registers, two threads per channel.  Lanes
+// 0-15 of a warp hold states 0 .. ceil(N/2)-1 of 16 channels and lanes 16-31 the other
+// states of the same channels; every sum over the states adds the two halves' partial
+// sums (lane ^ 16).  Half the registers per thread buys twice the warps per SM, which
+// hide the latency of the per-token loads.
+//   prologue: per token (split by parity between a channel's two threads), u, Delta and
+//     the output gradient through the gate, laid out time-major;
+//   forward sweep: every state's h_t (stored [B, L, N, D], so a warp's channels store one
+//     contiguous run per (token, state)) and the pre-gate output;
+//   reverse sweep: every state's adjoint, with h_t and h_(t-1) in registers and the next
+//     token's states and inputs loaded one step ahead;
+//   dB/dC: each token's contributions go to a shared buffer of kRedT tokens, summed over
+//     the tile's channels in channel order when it fills.
+// B and C of the sample are staged in shared memory as fp32 [t][2N].  A lane past the
+// tile's last channel computes on the tile's first channel and stores nothing, so every
+// lane takes part in the shuffles.
+constexpr int kFastN = 16, kHalfN = kFastN / 2, kRedT = 2;
 
 template <typename TI, typename TD, bool MIXER>
-__global__ void __launch_bounds__(64, 5) bwd_fast_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
   extern __shared__ float bsm[];
+  constexpr unsigned kAll = 0xffffffffu;
   const int tid = threadIdx.x, nthr = blockDim.x;
+  const int lane = tid & 31, half = lane >> 4;
+  const int cl = (tid >> 5) * 16 + (lane & 15);  // channel within the tile
   const int tile = blockIdx.x, b = blockIdx.y;
   const int d0 = tile * p.d_tile;
   const int dcount = min(p.d_tile, p.D - d0);
-  const bool active = tid < dcount;
-  const int d = d0 + (active ? tid : 0);
+  const bool active = cl < dcount;
+  const int d = d0 + (active ? cl : 0);
   const int L = p.L, N = p.N, N2 = 2 * p.N;
+  const int nh = (N + 1) / 2, n0 = half * nh, ncount = half ? N - nh : nh;  // this thread's states
   const bool gate = p.z != nullptr, use_sp = p.softplus;
   const size_t row = ((size_t)b * p.D + d) * L;
-  float* bc = bsm;                         // [L][2N]: B then C of token t
-  float* red = bsm + (size_t)L * N2;       // [kRedT][2N][d_tile + 1]
+  float* bc = bsm;                    // [L][2N]: B then C of token t
+  float* red = bsm + (size_t)L * N2;  // [kRedT][2N][d_tile + 1]
   const int rstride = p.d_tile + 1;
 
   const TI* u = MIXER ? nullptr : static_cast<const TI*>(p.u) + row;
@@ -223,9 +238,6 @@ __global__ void __launch_bounds__(64, 5) bwd_fast_kernel(const BwdParams p) {
   const TI* Cm = static_cast<const TI*>(p.Cm) + (size_t)b * N * L;
   const float dsk = p.Dskip ? p.Dskip[d] : 0.0f;
   const float dtb = p.dt_bias ? p.dt_bias[d] : 0.0f;
-  float* du = p.du + row;
-  float* ddt = p.ddt + row;
-  float* dz = gate ? p.dz + row : nullptr;
   const size_t tm0 = (size_t)b * L * p.D + d, tD = (size_t)p.D;
   float* tu = p.tm_u + tm0;
   float* tdl = p.tm_dl + tm0;
@@ -233,7 +245,8 @@ __global__ void __launch_bounds__(64, 5) bwd_fast_kernel(const BwdParams p) {
   float* tdu = p.tm_du + tm0;
   float* tdd = p.tm_dd + tm0;
   float* ty = p.tm_y + tm0;
-  float* hs = p.hstore + (size_t)b * L * N * p.D + d;  // h of (t, n) at hs[(t * N + n) * D]
+  // h of (t, state n0 + k) at hs[t * N * D + k * D]
+  float* hs = p.hstore + (size_t)b * L * N * p.D + (size_t)n0 * p.D + d;
 
   for (int e = tid; e < L * N2; e += nthr) {
     const int t = e / N2, j = e - t * N2;
@@ -247,77 +260,83 @@ __global__ void __launch_bounds__(64, 5) bwd_fast_kernel(const BwdParams p) {
     const int i = (MIXER && p.swap_dout) ? (t == 0 ? L - 1 : (t == L - 1 ? 0 : t)) : t;
     return to_f(dout[i]);
   };
+  // prologue: this thread's tokens t = half, half + 2, ...
   float sum_dsk = 0.0f;
-  if (active) {
+  {
     const TI* xr = MIXER ? static_cast<const TI*>(p.x) + ((size_t)b * p.D + d) * p.Tx : nullptr;
     float mean = 0.0f;
     if (MIXER && p.aux) {
-      for (int t = 0; t < p.Tx; ++t) mean += to_f(xr[t]);
-      mean /= (float)p.Tx;
+      float s = 0.0f;
+      for (int t = half; t < p.Tx; t += 2) s += to_f(xr[t]);
+      const float so = __shfl_xor_sync(kAll, s, 16);
+      mean = (half ? so + s : s + so) / (float)p.Tx;  // (even tokens) + (odd tokens) in both
     }
-#pragma unroll 2
-    for (int t = 0; t < L; ++t) {
+    for (int t = half; t < L; t += 2) {
       float ut;
       if constexpr (MIXER)
         ut = p.conv ? silu(conv_pre(p, xr, t, d, mean)) : xa_row(xr, t, L, p.aux, mean);
       else
         ut = to_f(u[t]);
       const float gy = gate ? dout_at(t) * silu(to_f(z[t])) : dout_at(t);
-      tu[t * tD] = ut;
-      tdl[t * tD] = delta_at(t);
-      tgy[t * tD] = gy;
-      tdu[t * tD] = gy * dsk;
-      tdd[t * tD] = 0.0f;
-      if (gate) ty[t * tD] = dsk * ut;
+      if (active) {
+        tu[t * tD] = ut;
+        tdl[t * tD] = delta_at(t);
+        tgy[t * tD] = gy;
+        tdu[t * tD] = gy * dsk;
+        tdd[t * tD] = 0.0f;
+        if (gate) ty[t * tD] = dsk * ut;
+      }
       sum_dsk = fmaf(gy, ut, sum_dsk);
     }
   }
   __syncthreads();
 
-  float An[kFastN];
+  float An[kHalfN];
 #pragma unroll
-  for (int n = 0; n < kFastN; ++n) An[n] = n < N ? p.A[(size_t)d * N + n] : 0.0f;
+  for (int k = 0; k < kHalfN; ++k) An[k] = k < ncount ? p.A[(size_t)d * N + n0 + k] : 0.0f;
+  const size_t hstep = (size_t)N * tD;  // h of the next token
 
-  // forward sweep: every state's h_t, and the pre-gate output for dz
-  if (active) {
-    float h[kFastN];
-    const size_t hstep = (size_t)N * tD;  // h of the next token
+  // forward sweep: this thread's states' h_t; the pre-gate output adds both halves
+  {
+    float h[kHalfN];
+#pragma unroll
+    for (int k = 0; k < kHalfN; ++k) h[k] = 0.0f;
     float* hp = hs;
-    const float* bt = bc;
-    // the next token's inputs are loaded one step ahead
+    const float* bt = bc + n0;  // B of state n0 + k at bt[k], its C at bt[N + k]
     float nd = tdl[0], nu = tu[0], ny = gate ? ty[0] : 0.0f;
     for (int t = 0; t < L; ++t, hp += hstep, bt += N2) {
-      const float delta = nd, ut = nu;
-      float yv = ny;
+      const float delta = nd, ut = nu, y0 = ny;
       if (t + 1 < L) {
         const size_t o = (size_t)(t + 1) * tD;
         nd = tdl[o];
         nu = tu[o];
         if (gate) ny = ty[o];
       }
+      float yp = 0.0f;
 #pragma unroll
-      for (int n = 0; n < kFastN; ++n) {
-        if (n < N) {
-          const float bu = delta * bt[n] * ut;
-          h[n] = t == 0 ? bu : fmaf(ex2(delta * An[n] * kLog2e), h[n], bu);
-          hp[n * tD] = h[n];
-          if (gate) yv = fmaf(bt[N + n], h[n], yv);
+      for (int k = 0; k < kHalfN; ++k) {
+        if (k < ncount) {
+          const float bu = delta * bt[k] * ut;
+          h[k] = t == 0 ? bu : fmaf(ex2(delta * An[k] * kLog2e), h[k], bu);
+          if (active) hp[k * tD] = h[k];
+          yp = fmaf(bt[N + k], h[k], yp);
         }
       }
-      if (gate) ty[(size_t)t * tD] = yv;
+      if (gate) {
+        const float yo = __shfl_xor_sync(kAll, yp, 16);
+        if (active && half == 0) ty[(size_t)t * tD] = y0 + (yp + yo);
+      }
     }
   }
 
-  // reverse sweep: every state's adjoint; the dB/dC contributions through the buffer
-  float g[kFastN], a_next[kFastN], dA[kFastN];
+  // reverse sweep: this thread's states' adjoints; du and dDelta add both halves
+  float g[kHalfN], a_next[kHalfN], dA[kHalfN];
 #pragma unroll
-  for (int n = 0; n < kFastN; ++n) g[n] = a_next[n] = dA[n] = 0.0f;
+  for (int k = 0; k < kHalfN; ++k) g[k] = a_next[k] = dA[k] = 0.0f;
   const size_t pbc = (((size_t)b * p.ntiles + tile) * 2) * N * L;
-  const size_t hstep = (size_t)N * tD;
-  // h_t and h_(t-1) are in registers; h_(t-2) and the next token's inputs load one step ahead
-  float hc[kFastN], hq[kFastN];
-  float nd = 0.0f, ngy = 0.0f, nu = 0.0f, ndu = 0.0f, ndd = 0.0f;
-  if (active) {
+  float hc[kHalfN], hq[kHalfN];  // h_t and h_(t-1); h_(t-2) and the next inputs load one step ahead
+  float nd, ngy, nu, ndu, ndd;
+  {
     const size_t o = (size_t)(L - 1) * tD;
     nd = tdl[o];
     ngy = tgy[o];
@@ -325,57 +344,58 @@ __global__ void __launch_bounds__(64, 5) bwd_fast_kernel(const BwdParams p) {
     ndu = tdu[o];
     ndd = tdd[o];
 #pragma unroll
-    for (int n = 0; n < kFastN; ++n) {
-      hc[n] = n < N ? hs[(size_t)(L - 1) * hstep + n * tD] : 0.0f;
-      hq[n] = (n < N && L > 1) ? hs[(size_t)(L - 2) * hstep + n * tD] : 0.0f;
+    for (int k = 0; k < kHalfN; ++k) {
+      hc[k] = k < ncount ? hs[(size_t)(L - 1) * hstep + k * tD] : 0.0f;
+      hq[k] = (k < ncount && L > 1) ? hs[(size_t)(L - 2) * hstep + k * tD] : 0.0f;
     }
   }
   for (int t = L - 1; t >= 0; --t) {
     const int slot = (L - 1 - t) % kRedT;
-    if (active) {
-      const size_t o = (size_t)t * tD;
-      const float delta = nd, gy = ngy, ut = nu;
-      float duv = ndu, ddv = ndd;
-      float hn[kFastN];  // h_(t-2), for the next step
-      if (t >= 1) {
-        const size_t o1 = (size_t)(t - 1) * tD;
-        nd = tdl[o1];
-        ngy = tgy[o1];
-        nu = tu[o1];
-        ndu = tdu[o1];
-        ndd = tdd[o1];
-      }
+    const float delta = nd, gy = ngy, ut = nu, du0 = ndu, dd0 = ndd;
+    if (t >= 1) {
+      const size_t o1 = (size_t)(t - 1) * tD;
+      nd = tdl[o1];
+      ngy = tgy[o1];
+      nu = tu[o1];
+      ndu = tdu[o1];
+      ndd = tdd[o1];
+    }
+    float hn[kHalfN];  // h_(t-2), for the next step
 #pragma unroll
-      for (int n = 0; n < kFastN; ++n) hn[n] = (n < N && t >= 2) ? hs[(size_t)(t - 2) * hstep + n * tD] : 0.0f;
-      const float* bt = bc + (size_t)t * N2;
-      float* rs = red + (size_t)slot * N2 * rstride + tid;
+    for (int k = 0; k < kHalfN; ++k) hn[k] = (k < ncount && t >= 2) ? hs[(size_t)(t - 2) * hstep + k * tD] : 0.0f;
+    const float* bt = bc + (size_t)t * N2 + n0;
+    float* rs = red + (size_t)slot * N2 * rstride + (size_t)n0 * rstride + cl;
+    float dup = 0.0f, ddp = 0.0f;
 #pragma unroll
-      for (int n = 0; n < kFastN; ++n) {
-        if (n < N) {
-          const float Bv = bt[n], Cv = bt[N + n];
-          g[n] = fmaf(gy, Cv, t + 1 < L ? a_next[n] * g[n] : 0.0f);
-          rs[(N + n) * rstride] = gy * hc[n];
-          rs[n * rstride] = g[n] * delta * ut;
-          duv = fmaf(g[n] * delta, Bv, duv);
-          float dd = g[n] * Bv * ut;
-          float a_t = 0.0f;
-          if (t > 0) {
-            a_t = ex2(delta * An[n] * kLog2e);
-            const float gha = g[n] * hq[n] * a_t;
-            dd = fmaf(gha, An[n], dd);
-            dA[n] = fmaf(gha, delta, dA[n]);
-          }
-          ddv += dd;
-          a_next[n] = a_t;
+    for (int k = 0; k < kHalfN; ++k) {
+      if (k < ncount) {
+        const float Bv = bt[k], Cv = bt[N + k];
+        g[k] = fmaf(gy, Cv, t + 1 < L ? a_next[k] * g[k] : 0.0f);
+        rs[(N + k) * rstride] = gy * hc[k];
+        rs[k * rstride] = g[k] * delta * ut;
+        dup = fmaf(g[k] * delta, Bv, dup);
+        float dd = g[k] * Bv * ut;
+        float a_t = 0.0f;
+        if (t > 0) {
+          a_t = ex2(delta * An[k] * kLog2e);
+          const float gha = g[k] * hq[k] * a_t;
+          dd = fmaf(gha, An[k], dd);
+          dA[k] = fmaf(gha, delta, dA[k]);
         }
+        ddp += dd;
+        a_next[k] = a_t;
       }
-      tdu[o] = duv;
-      tdd[o] = ddv;
+    }
+    const float dupo = __shfl_xor_sync(kAll, dup, 16), ddpo = __shfl_xor_sync(kAll, ddp, 16);
+    if (active && half == 0) {
+      const size_t o = (size_t)t * tD;
+      tdu[o] = du0 + (dup + dupo);
+      tdd[o] = dd0 + (ddp + ddpo);
+    }
 #pragma unroll
-      for (int n = 0; n < kFastN; ++n) {
-        hc[n] = hq[n];
-        hq[n] = hn[n];
-      }
+    for (int k = 0; k < kHalfN; ++k) {
+      hc[k] = hq[k];
+      hq[k] = hn[k];
     }
     if (slot == kRedT - 1 || t == 0) {  // the buffered tokens t .. t + slot: sum over channels in order
       __syncthreads();
@@ -391,30 +411,37 @@ __global__ void __launch_bounds__(64, 5) bwd_fast_kernel(const BwdParams p) {
     }
   }
 
-  if (active) {
+  // epilogue: this thread's tokens; the last barrier above ordered every tdu/tdd write
+  if (active)
 #pragma unroll
-    for (int n = 0; n < kFastN; ++n)
-      if (n < N) p.partA[((size_t)b * p.D + d) * N + n] = dA[n];
-    float sum_bias = 0.0f;
-#pragma unroll 4
-    for (int t = 0; t < L; ++t) {
-      const float v = to_f(dt[t]) + dtb;
-      const float dd = tdd[t * tD];
-      const float ds = use_sp ? dd * (v > 20.0f ? 1.0f : sigmoid(v)) : dd;
+    for (int k = 0; k < kHalfN; ++k)
+      if (k < ncount) p.partA[((size_t)b * p.D + d) * N + n0 + k] = dA[k];
+  float* du = p.du + row;
+  float* ddt = p.ddt + row;
+  float* dz = gate ? p.dz + row : nullptr;
+  float sum_bias = 0.0f;
+  for (int t = half; t < L; t += 2) {
+    const float v = to_f(dt[t]) + dtb;
+    const float dd = tdd[t * tD];
+    const float ds = use_sp ? dd * (v > 20.0f ? 1.0f : sigmoid(v)) : dd;
+    if (active) {
       ddt[t] = ds;
       du[t] = tdu[t * tD];
-      sum_bias += ds;
       if (gate) {
         const float zt = to_f(z[t]), sg = sigmoid(zt);
         dz[t] = dout_at(t) * ty[t * tD] * (sg * (1.0f + zt * (1.0f - sg)));
       }
     }
-    p.partD[(size_t)b * p.D + d] = sum_dsk;
-    p.partBias[(size_t)b * p.D + d] = sum_bias;
+    sum_bias += ds;
+  }
+  const float sdo = __shfl_xor_sync(kAll, sum_dsk, 16), sbo = __shfl_xor_sync(kAll, sum_bias, 16);
+  if (active && half == 0) {
+    p.partD[(size_t)b * p.D + d] = sum_dsk + sdo;
+    p.partBias[(size_t)b * p.D + d] = sum_bias + sbo;
   }
 }
 
-// The register-resident kernel covers N <= 16 with B and C of a sample in 64 KB of
+// The register-resident kernels cover N <= 16 with B and C of a sample in 64 KB of
 // shared memory; other shapes take bwd_main_kernel.
 static bool bwd_fast_ok(int N, int L, int d_tile) {
   return N <= kFastN && d_tile <= 64 && bwd_fast_smem(N, L, d_tile) <= 64 * 1024;
@@ -522,12 +549,12 @@ cudaError_t noalloc_scratch(void** out) {
 template <typename TI, typename TD, bool MIXER>
 static cudaError_t launch_main(const BwdParams& p, cudaStream_t s) {
   const int threads = (p.d_tile + 31) & ~31;
-  if (p.hstore) {
+  if (p.hstore) {  // two threads per channel, 16 channels per warp
     const int bytes = bwd_fast_smem(p.N, p.L, p.d_tile);
     static SmemLimit lim;
-    cudaError_t e = raise_smem_limit(bwd_fast_kernel<TI, TD, MIXER>, bytes, lim);
+    cudaError_t e = raise_smem_limit(bwd_pair_kernel<TI, TD, MIXER>, bytes, lim);
     if (e != cudaSuccess) return e;
-    bwd_fast_kernel<TI, TD, MIXER><<<dim3(p.ntiles, p.B), threads, bytes, s>>>(p);
+    bwd_pair_kernel<TI, TD, MIXER><<<dim3(p.ntiles, p.B), 2 * ((p.d_tile + 15) & ~15), bytes, s>>>(p);
   } else {
     bwd_main_kernel<TI, TD, MIXER><<<dim3(p.ntiles, p.B), threads, 0, s>>>(p);
   }
