@@ -282,8 +282,6 @@ __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
         tu[t * tD] = ut;
         tdl[t * tD] = delta_at(t);
         tgy[t * tD] = gy;
-        tdu[t * tD] = gy * dsk;
-        tdd[t * tD] = 0.0f;
         if (gate) ty[t * tD] = dsk * ut;
       }
       sum_dsk = fmaf(gy, ut, sum_dsk);
@@ -335,14 +333,12 @@ __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
   for (int k = 0; k < kHalfN; ++k) g[k] = a_next[k] = dA[k] = 0.0f;
   const size_t pbc = (((size_t)b * p.ntiles + tile) * 2) * N * L;
   float hc[kHalfN], hq[kHalfN];  // h_t and h_(t-1); h_(t-2) and the next inputs load one step ahead
-  float nd, ngy, nu, ndu, ndd;
+  float nd, ngy, nu;
   {
     const size_t o = (size_t)(L - 1) * tD;
     nd = tdl[o];
     ngy = tgy[o];
     nu = tu[o];
-    ndu = tdu[o];
-    ndd = tdd[o];
 #pragma unroll
     for (int k = 0; k < kHalfN; ++k) {
       hc[k] = k < ncount ? hs[(size_t)(L - 1) * hstep + k * tD] : 0.0f;
@@ -351,14 +347,12 @@ __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
   }
   for (int t = L - 1; t >= 0; --t) {
     const int slot = (L - 1 - t) % kRedT;
-    const float delta = nd, gy = ngy, ut = nu, du0 = ndu, dd0 = ndd;
+    const float delta = nd, gy = ngy, ut = nu;
     if (t >= 1) {
       const size_t o1 = (size_t)(t - 1) * tD;
       nd = tdl[o1];
       ngy = tgy[o1];
       nu = tu[o1];
-      ndu = tdu[o1];
-      ndd = tdd[o1];
     }
     float hn[kHalfN];  // h_(t-2), for the next step
 #pragma unroll
@@ -387,10 +381,10 @@ __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
       }
     }
     const float dupo = __shfl_xor_sync(kAll, dup, 16), ddpo = __shfl_xor_sync(kAll, ddp, 16);
-    if (active && half == 0) {
+    if (active && half == 0) {  // du_t = dy_t Dskip + the states' share; dDelta_t = the states' share
       const size_t o = (size_t)t * tD;
-      tdu[o] = du0 + (dup + dupo);
-      tdd[o] = dd0 + (ddp + ddpo);
+      tdu[o] = fmaf(gy, dsk, dup + dupo);
+      tdd[o] = ddp + ddpo;
     }
 #pragma unroll
     for (int k = 0; k < kHalfN; ++k) {
