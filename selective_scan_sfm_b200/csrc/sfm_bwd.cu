@@ -45,9 +45,14 @@ __device__ __forceinline__ float conv_pre(const BwdParams& p, const TI* xr, int 
   return acc;
 }
 
+// Register-resident backward: states per channel at most, states per thread, tokens per
+// dB/dC buffer, and the buffer's rows per token (B and C of each half's kHalfN states).
+constexpr int kFastN = 16, kHalfN = kFastN / 2, kRedT = 2, kRedRows = 2 * kFastN;
+
 static int bwd_fast_smem(int N, int L, int d_tile) {
-  // bc [L][2N] + red: 2 tokens x 2N rows of d_tile + 1 (the pad keeps the row sums off one bank)
-  return (int)(((size_t)L * 2 * N + (size_t)2 * 2 * N * (d_tile + 1)) * sizeof(float));
+  // bc [L][2N] + red: kRedT tokens x kRedRows rows of d_tile + 1 (the pad keeps the row sums
+  // off one bank)
+  return (int)(((size_t)L * 2 * N + (size_t)kRedT * kRedRows * (d_tile + 1)) * sizeof(float));
 }
 
 template <typename TI, typename TD, bool MIXER>
@@ -208,7 +213,6 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
 // B and C of the sample are staged in shared memory as fp32 [t][2N].  A lane past the
 // tile's last channel computes on the tile's first channel and stores nothing, so every
 // lane takes part in the shuffles.
-constexpr int kFastN = 16, kHalfN = kFastN / 2, kRedT = 2;
 
 template <typename TI, typename TD, bool MIXER>
 __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
@@ -227,7 +231,9 @@ __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
   const bool gate = p.z != nullptr, use_sp = p.softplus;
   const size_t row = ((size_t)b * p.D + d) * L;
   float* bc = bsm;                    // [L][2N]: B then C of token t
-  float* red = bsm + (size_t)L * N2;  // [kRedT][2N][d_tile + 1]
+  // [kRedT][kRedRows][d_tile + 1]: half h's B rows at 16h .. 16h+7, its C rows at 16h+8 ..
+  // 16h+15, so the two halves' stores of one state index land 16 banks apart
+  float* red = bsm + (size_t)L * N2;
   const int rstride = p.d_tile + 1;
 
   const TI* u = MIXER ? nullptr : static_cast<const TI*>(p.u) + row;
@@ -358,14 +364,14 @@ __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
 #pragma unroll
     for (int k = 0; k < kHalfN; ++k) hn[k] = (k < ncount && t >= 2) ? hs[(size_t)(t - 2) * hstep + k * tD] : 0.0f;
     const float* bt = bc + (size_t)t * N2 + n0;
-    float* rs = red + (size_t)slot * N2 * rstride + (size_t)n0 * rstride + cl;
+    float* rs = red + ((size_t)slot * kRedRows + 2 * kHalfN * half) * rstride + cl;
     float dup = 0.0f, ddp = 0.0f;
 #pragma unroll
     for (int k = 0; k < kHalfN; ++k) {
       if (k < ncount) {
         const float Bv = bt[k], Cv = bt[N + k];
         g[k] = fmaf(gy, Cv, t + 1 < L ? a_next[k] * g[k] : 0.0f);
-        rs[(N + k) * rstride] = gy * hc[k];
+        rs[(kHalfN + k) * rstride] = gy * hc[k];
         rs[k * rstride] = g[k] * delta * ut;
         dup = fmaf(g[k] * delta, Bv, dup);
         float dd = g[k] * Bv * ut;
@@ -393,13 +399,16 @@ __global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
     }
     if (slot == kRedT - 1 || t == 0) {  // the buffered tokens t .. t + slot: sum over channels in order
       __syncthreads();
-      for (int e = tid; e < (slot + 1) * N2; e += nthr) {
-        const int k = e / N2, j = e - k * N2;  // buffer slot k holds token t + slot - k
-        const float* r = red + ((size_t)k * N2 + j) * rstride;
+      for (int e = tid; e < (slot + 1) * kRedRows; e += nthr) {
+        const int k = e / kRedRows, j = e - k * kRedRows;  // buffer slot k holds token t + slot - k
+        const int hh = j / (2 * kHalfN), kk = j % kHalfN, n = hh * nh + kk;
+        const bool is_c = (j / kHalfN) & 1;
+        if (kk >= (hh ? N - nh : nh)) continue;  // a row of no state
+        const float* r = red + ((size_t)k * kRedRows + j) * rstride;
         float sum = 0.0f;
         for (int c = 0; c < dcount; ++c) sum += r[c];
         const int tt = t + slot - k;
-        p.partBC[pbc + (j < N ? (size_t)j * L : (size_t)N * L + (size_t)(j - N) * L) + tt] = sum;
+        p.partBC[pbc + (is_c ? (size_t)N * L : 0) + (size_t)n * L + tt] = sum;
       }
       __syncthreads();
     }
