@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(128) bwd_main_kernel(const BwdParams p) {
 // lane takes part in the shuffles.
 
 template <typename TI, typename TD, bool MIXER>
-__global__ void __launch_bounds__(128, 4) bwd_pair_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(128, MIXER ? 5 : 4) bwd_pair_kernel(const BwdParams p) {
   extern __shared__ float bsm[];
   constexpr unsigned kAll = 0xffffffffu;
   const int tid = threadIdx.x, nthr = blockDim.x;
