@@ -172,3 +172,22 @@ def test_backward_large_state_size():
     d2 = synth.make_inputs(B=2, D=40, T=30, N=32, dtype="f32", seed=4301, random_A=True)
     g2, ref2 = run_mixer_both(d2, synth.make_dout(2, 40, 32, seed=4301, dtype="f32"), True, True)
     check_mixer(g2, ref2, TOL["f32"])
+
+
+@pytest.mark.parametrize("N", [1, 3, 5, 15])
+def test_backward_odd_state_sizes(N):
+    """Odd N splits the states unequally between a channel's two threads (the second half
+    one state short, empty at N = 1); D = 70 leaves a partial last channel tile."""
+    d = synth.make_inputs(B=3, D=70, T=37, N=N, dtype="f32", seed=4400 + N, aux=False, random_A=True)
+    dout = synth.make_dout(3, 70, 37, seed=4400 + N, dtype="f32")
+    g, ref = run_both(d, dout)
+    check_grads(g, ref, TOL["f32"], TOL["f32"])
+
+
+@pytest.mark.parametrize("N", [1, 7])
+def test_mixer_backward_odd_state_sizes(N):
+    B, D, T = 2, 70, 33
+    d = synth.make_inputs(B=B, D=D, T=T, N=N, dtype="f32", seed=4500 + N, random_A=True)
+    dout = synth.make_dout(B, D, T + 2, seed=4500 + N, dtype="f32")
+    g, ref = run_mixer_both(d, dout, True, True, 1, True)
+    check_mixer(g, ref, TOL["f32"])
