@@ -11,7 +11,9 @@ table.  Prints one JSON line on rank 0.
   timed with CUDA events on the launch stream between a barrier + synchronize on both
   sides, max over ranks.  Inputs rotate over several sets whose total exceeds 2x L2.
 * e2e: the same metric through the public Python API with each step's inputs copied
-  host->device from pinned memory and the output read back device->host.
+  host->device from pinned memory and the output read back device->host; two device
+  buffer sets on three streams let one step's upload overlap the previous step's kernel
+  and readback.
 * roofline: the kernel is bound by its transcendental arithmetic (MUFU), not by HBM;
   the ALU peak is derived from unit counts and the SM clock; the HBM
   fraction is reported next to it.
@@ -322,34 +324,63 @@ def measure(workload, steps, warmup, world, rank, device, seed_base=0, with_e2e=
                elements=B * D * L, bytes=set_bytes, variant=var, nsets=nsets, set_bytes=set_bytes, w=w, L=L)
 
     if with_e2e:
-        # the public API with host buffers: pinned H2D of the step's inputs, D2H of y
+        # the public API with host buffers: pinned H2D of the step's inputs, D2H of y.  Two
+        # device buffer sets on three streams: step i+1's H2D overlaps step i's kernel and
+        # D2H (PCIe carries both directions at once); each step still copies its own inputs
+        # in and its own output out inside the timed region.
         host = synth.make_inputs(**w, seed=seed_base + 999)
         pin = {k: host[k].pin_memory() for k in ("x", "dt", "z", "Bm", "Cm")}
-        dev = {k: torch.empty_like(pin[k], device=device) for k in pin}
         par = {k: host[k].to(device) for k in ("A", "Dskip", "dt_bias", "conv_w", "conv_b")}
-        yh = torch.empty(B, D, L, dtype=io).pin_memory()
-        yd = torch.empty(B, D, L, dtype=io, device=device)
+        dev = [{k: torch.empty_like(pin[k], device=device) for k in pin} for _ in range(2)]
+        yd = [torch.empty(B, D, L, dtype=io, device=device) for _ in range(2)]
+        yh = [torch.empty(B, D, L, dtype=io).pin_memory() for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in pin.values())
-        d2h = yh.numel() * yh.element_size()
+        d2h = yh[0].numel() * yh[0].element_size()
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev = lambda: torch.cuda.Event()
+        in_done, run_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+        used = [False, False]
 
-        def e2e_step():
-            for k in pin:
-                dev[k].copy_(pin[k], non_blocking=True)
-            sfm_selective_scan_fold(dev["x"], dev["dt"], dev["Bm"], dev["Cm"], par["A"], z=dev["z"],
+        def e2e_step(i):
+            j = i % 2
+            with torch.cuda.stream(s_in):
+                if used[j]:
+                    s_in.wait_event(run_done[j])   # the kernel two steps back has read dev[j]
+                for k in pin:
+                    dev[j][k].copy_(pin[k], non_blocking=True)
+                in_done[j].record(s_in)
+            stream.wait_event(in_done[j])
+            if used[j]:
+                stream.wait_event(out_done[j])     # yd[j] has been read out
+            sfm_selective_scan_fold(dev[j]["x"], dev[j]["dt"], dev[j]["Bm"], dev[j]["Cm"], par["A"], z=dev[j]["z"],
                                     Dskip=par["Dskip"], dt_bias=par["dt_bias"], conv_w=par["conv_w"],
-                                    conv_b=par["conv_b"], y=yd, aux_init=True)
-            yh.copy_(yd, non_blocking=True)
+                                    conv_b=par["conv_b"], y=yd[j], aux_init=True)
+            run_done[j].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(run_done[j])
+                yh[j].copy_(yd[j], non_blocking=True)
+                out_done[j].record(s_out)
+            used[j] = True
+
+        def drain():  # the launch stream waits for every copy in flight
+            for j in range(2):
+                if used[j]:
+                    stream.wait_event(out_done[j])
 
         e2e_steps = max(3, min(steps, 20))
-        for _ in range(3):
-            e2e_step()
+        for i in range(3):
+            e2e_step(i)
+        drain()
         torch.cuda.synchronize(device)
         if world > 1:
             torch.distributed.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        drain()
         e1.record(stream)
         torch.cuda.synchronize(device)
         if world > 1:
@@ -678,7 +709,9 @@ def main(argv=None):
                 "peak_source": peak_src, "algorithmic_bytes_per_launch": res["bytes"]},
         "kernel_ms": launch_ms,
         "e2e": {"value": e2e_value, "unit": "elems/s", "h2d_bytes_per_step": res["h2d"],
-                "d2h_bytes_per_step": res["d2h"]},
+                "d2h_bytes_per_step": res["d2h"],
+                "schedule": "two device buffer sets; H2D, kernel and D2H on three streams, so step i+1's "
+                            "H2D overlaps step i's kernel and D2H"},
         "gpu_launches": args.steps,  # timed region of the main workload: one kernel per step
         "clocks": ck,
     }
